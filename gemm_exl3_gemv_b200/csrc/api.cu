@@ -1,0 +1,161 @@
+// api.cu -- the extern "C" entry points of libexl3 (declared in include/exl3.h):
+// argument validation on the host, architecture check, dispatch to kernels.
+#include <cstdint>
+#include <cstring>
+
+#include "../../include/exl3.h"
+#include "exl3_common.cuh"
+#include "exl3_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+int cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = (int)e;
+    return EXL3_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4; }
+
+// The kernels are built for sm_100a only; check the current device once per
+// call (cheap: cached attribute queries in the runtime).
+int check_arch()
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    int major = 0, minor = 0;
+    e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return (major == 10 && minor == 0) ? EXL3_OK : EXL3_ERR_ARCH;
+}
+
+int validate_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale, const uint16_t* su,
+                  const uint16_t* sv, const void* y, int k_in, int n_out, int bits, const void* ws, size_t ws_bytes)
+{
+    if (!x || !packed || !scale || !su || !sv || !y) return EXL3_ERR_INVALID_ARG;
+    if (m <= 0 || k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
+    if (m > 32 || !bits_ok(bits) || k_in % 128 || n_out % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(su) || !aligned16(sv) ||
+        !aligned16(y))
+        return EXL3_ERR_MISALIGNED;
+    if (!ws || ws_bytes < exl3_workspace_bytes(m, k_in, n_out, bits)) return EXL3_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return EXL3_ERR_MISALIGNED;
+    return EXL3_OK;
+}
+
+int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale, const uint16_t* su,
+             const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out, int bits, void* ws, size_t ws_bytes,
+             void* stream)
+{
+    int st = validate_gemm(m, x, packed, scale, su, sv, y, k_in, n_out, bits, ws, ws_bytes);
+    if (st != EXL3_OK) return st;
+    st = check_arch();
+    if (st != EXL3_OK) return st;
+    exl3::GemmArgs a;
+    a.x = x;
+    a.packed = packed;
+    a.scale = scale;
+    a.su = su;
+    a.sv = sv;
+    a.y = y;
+    a.y_fp32 = y_fp32 ? 1 : 0;
+    a.m = m;
+    a.k_in = k_in;
+    a.n_out = n_out;
+    a.bits = bits;
+    a.ws = static_cast<unsigned char*>(ws);
+    cudaError_t e = exl3::launch_gemv_cc(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* exl3_status_string(int status)
+{
+    switch (status) {
+        case EXL3_OK: return "EXL3_OK";
+        case EXL3_ERR_INVALID_ARG: return "EXL3_ERR_INVALID_ARG: null pointer, non-positive size or bad mode";
+        case EXL3_ERR_UNSUPPORTED: return "EXL3_ERR_UNSUPPORTED: bits, shape or row count not supported";
+        case EXL3_ERR_MISALIGNED: return "EXL3_ERR_MISALIGNED: pointer not 16-byte (workspace: 256-byte) aligned";
+        case EXL3_ERR_WORKSPACE: return "EXL3_ERR_WORKSPACE: workspace missing or too small";
+        case EXL3_ERR_ARCH: return "EXL3_ERR_ARCH: current device is not a compute capability 10.0 GPU";
+        case EXL3_ERR_CUDA: return "EXL3_ERR_CUDA: a CUDA runtime call failed (see exl3_last_cuda_error)";
+        case EXL3_ERR_TIMEOUT: return "EXL3_ERR_TIMEOUT: a kernel gave up a bounded wait; output invalid";
+    }
+    return "EXL3: unknown status";
+}
+
+int exl3_last_cuda_error(void) { return g_last_cuda_error; }
+
+int exl3_version(void) { return 100; }
+
+size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits)
+{
+    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
+    return exl3::cc_workspace_bytes(m, k_in, n_out, bits);
+}
+
+int exl3_workspace_status(void* workspace, void* stream)
+{
+    if (!workspace) return EXL3_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t word = 0;
+    cudaError_t e = cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (word == 0) return EXL3_OK;
+    e = cudaMemsetAsync(workspace, 0, sizeof(word), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return EXL3_ERR_TIMEOUT;
+}
+
+int exl3_decode_tiles(const uint32_t* packed, int k_in, int n_out, int bits, uint16_t* w_out, void* stream)
+{
+    if (!packed || !w_out || k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
+    if (!bits_ok(bits) || k_in % 16 || n_out % 16) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(packed) || !aligned16(w_out)) return EXL3_ERR_MISALIGNED;
+    int st = check_arch();
+    if (st != EXL3_OK) return st;
+    cudaError_t e = exl3::launch_decode_tiles(packed, k_in, n_out, bits, w_out, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
+int exl3_hadamard128(const uint16_t* in, uint16_t* out, const uint16_t* signs, int rows, int n, int mode,
+                     void* stream)
+{
+    if (!in || !out || !signs || rows <= 0 || n <= 0 || (mode != 0 && mode != 1)) return EXL3_ERR_INVALID_ARG;
+    if (n % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(in) || !aligned16(out) || !aligned16(signs)) return EXL3_ERR_MISALIGNED;
+    int st = check_arch();
+    if (st != EXL3_OK) return st;
+    cudaError_t e = exl3::launch_hadamard128(in, out, signs, rows, n, mode, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
+int exl3_gemv(const uint16_t* x, const uint32_t* packed, const uint16_t* scale, const uint16_t* su,
+              const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out, int bits, void* workspace,
+              size_t ws_bytes, void* stream)
+{
+    return run_gemm(1, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, workspace, ws_bytes, stream);
+}
+
+int exl3_gemm_small_m(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale, const uint16_t* su,
+                      const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out, int bits, void* workspace,
+                      size_t ws_bytes, void* stream)
+{
+    return run_gemm(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, workspace, ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,129 @@
+// exl3_common.cuh -- helpers shared by the libexl3 kernels: shared-memory
+// barriers and bulk copies (sm_90+ PTX), the warp-level Hadamard-128, and the
+// workspace layout.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace exl3 {
+
+// ------------------------------------------------------------ workspace ---
+// [0, 256)            status word (uint32 at 0): nonzero after a timed-out wait
+// [256, 256 + 4*G)    one arrival counter per 128-channel output block
+// [ws_part_off, ...)  split-K partial sums, fp32 [splits][m][n_out]
+constexpr size_t kWsHeader = 256;
+constexpr uint32_t kStatusTimeout = 1u;
+
+__host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+__host__ __device__ inline size_t ws_counter_off() { return kWsHeader; }
+__host__ __device__ inline size_t ws_part_off(int n_out) { return align_up(kWsHeader + 4 * (size_t)(n_out / 128), 256); }
+
+// ------------------------------------------------------------ addressing ---
+__device__ __forceinline__ uint32_t smem_u32(const void* p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ------------------------------------------------------------- mbarrier ---
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// make barrier initialisation visible to the async (bulk-copy) proxy
+__device__ __forceinline__ void fence_mbar_init()
+{
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for phase `parity` of `bar` to complete, giving up after ~`limit_ns`
+// nanoseconds.  Returns false on timeout (the caller records it and skips
+// its work; nothing spins forever).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns = 2000000000ull)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        for (int i = 0; i < 64; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
+        if (global_ns() - t0 > limit_ns) return false;
+    }
+}
+
+// 1-D bulk copy global -> shared, completion reported on `bar` (tx bytes).
+// dst, src 16-byte aligned; bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// ------------------------------------------------------------ Hadamard ---
+// Unnormalised Walsh-Hadamard transform of one 128-element block held by a
+// warp, 4 consecutive elements per lane (element 4*lane + e in v[e]).  Natural
+// (Sylvester) order: butterflies (a, b) -> (a + b, a - b) with `a` the element
+// whose index has the stage bit clear.
+__device__ __forceinline__ void fwht128_warp(float (&v)[4])
+{
+    // stage bits 0 and 1 are inside the lane
+    float a0 = v[0] + v[1], a1 = v[0] - v[1], a2 = v[2] + v[3], a3 = v[2] - v[3];
+    v[0] = a0 + a2;
+    v[1] = a1 + a3;
+    v[2] = a0 - a2;
+    v[3] = a1 - a3;
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {      // stage bits 2..6 live in the lane index
+        const bool upper = (lane & d) != 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[e], d);
+            v[e] = upper ? (p - v[e]) : (v[e] + p);
+        }
+    }
+}
+
+constexpr float kInvSqrt128 = 0.08838834764831845f;
+
+}  // namespace exl3

@@ -1,0 +1,32 @@
+// exl3_internal.h -- launchers shared between the libexl3 translation units.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace exl3 {
+
+cudaError_t launch_decode_tiles(const uint32_t* packed, int k_in, int n_out, int bits, uint16_t* w_out,
+                                cudaStream_t stream);
+cudaError_t launch_hadamard128(const uint16_t* in, uint16_t* out, const uint16_t* signs, int rows, int n, int mode,
+                               cudaStream_t stream);
+
+// Problem description shared by the product kernels.
+struct GemmArgs {
+    const uint16_t* x;        // m x k_in fp16
+    const uint32_t* packed;   // trellis words
+    const uint16_t* scale;    // n_out fp16
+    const uint16_t* su;       // k_in fp16 +-1
+    const uint16_t* sv;       // n_out fp16 +-1
+    void* y;                  // m x n_out, fp16 or fp32
+    int y_fp32;
+    int m, k_in, n_out, bits;
+    unsigned char* ws;        // workspace base
+};
+
+// Split-K factor the CUDA-core kernel uses for this problem (host-only).
+int cc_splits(int m, int k_in, int n_out, int bits);
+size_t cc_workspace_bytes(int m, int k_in, int n_out, int bits);
+cudaError_t launch_gemv_cc(const GemmArgs& a, cudaStream_t stream);
+
+}  // namespace exl3

@@ -1,0 +1,158 @@
+/*
+ * exl3.h -- C ABI of libexl3: matrix-vector and skinny-matrix products
+ * against EXL3-style trellis-quantised weights on NVIDIA B200 (sm_100a).
+ *
+ * What is computed.  The pages this library follows name the EXL3 trellis
+ * format and its decode-time GEMV without defining it ("~3.2 bits/weight in
+ * the EXL3 trellis format", orcasaq2-rocm README, opening paragraph; "EXL3
+ * GEMM kernels were rewritten for RDNA's vector ALUs", same page, second
+ * paragraph; "checking 8 drafted tokens", "batched verification up to 32
+ * rows", exl3-rdna4-recipe, section "What we added on top of upstream").  The
+ * format fixed here:
+ *   - W is K_in x N_out, stored as 16x16 tiles; tile (tk, tn) is tile number
+ *     tk*(N_out/16) + tn and holds 8*K uint32 words (K = bits per weight) that
+ *     form one tail-biting bitstream of 256*K bits.  Stream bit j is bit
+ *     31-(j%32) of word j/32 (most significant bit first).
+ *   - weight i of a tile (row i/16, column i%16 of the tile) is decoded from
+ *     the 16 stream bits ending at bit (i+1)*K (positions modulo 256*K; the
+ *     earliest bit is the most significant) with the 3INST map
+ *         x = state*89226354 + 64248484  (mod 2^32)
+ *         m = (x & 0x8FFF8FFF) ^ 0x3B603B60
+ *         w = fp16(m[15:0]) + fp16(m[31:16])   (one rounding to fp16, RNE)
+ *   - y = sv .* H( scale .* ( H(su .* x) W ) ), where H is the normalised
+ *     128-point Hadamard transform (Sylvester order, entries
+ *     (-1)^popcount(i&j)/sqrt(128)) applied to each contiguous 128-element
+ *     block, su (K_in) and sv (N_out) are +-1 sign vectors and scale (N_out)
+ *     is a per-output-channel fp16 scale.
+ *
+ * Conventions shared by every entry point.
+ *   - All array arguments are DEVICE pointers (cudaMalloc / PyTorch CUDA
+ *     memory) owned by the caller; the library allocates nothing, frees
+ *     nothing and never synchronises the stream.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued on it and the call returns.
+ *   - fp16 arrays are passed as uint16_t bit patterns (IEEE binary16).
+ *   - Every pointer must be 16-byte aligned (EXL3_ERR_MISALIGNED otherwise).
+ *   - Arguments are validated on the host before anything is enqueued; an
+ *     invalid call returns its status and enqueues nothing.  A CUDA launch
+ *     failure returns EXL3_ERR_CUDA (exl3_last_cuda_error() gives the
+ *     cudaError_t).  Faults inside a kernel surface, CUDA-style, at the
+ *     caller's next synchronisation.
+ *   - The device current on the calling thread must be a B200 (compute
+ *     capability 10.0); otherwise EXL3_ERR_ARCH.
+ */
+#ifndef EXL3_H
+#define EXL3_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define EXL3_API __attribute__((visibility("default")))
+#else
+#define EXL3_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    EXL3_OK = 0,
+    EXL3_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad mode     */
+    EXL3_ERR_UNSUPPORTED = 2,  /* bits not in {2,3,4}; shape not a multiple of
+                                  128 (16 for decode); m outside [1, 32]        */
+    EXL3_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned               */
+    EXL3_ERR_WORKSPACE = 4,    /* workspace null or smaller than required        */
+    EXL3_ERR_ARCH = 5,         /* current device is not compute capability 10.0 */
+    EXL3_ERR_CUDA = 6,         /* a CUDA runtime call failed                     */
+    EXL3_ERR_TIMEOUT = 7       /* a kernel's bounded wait expired (see
+                                  exl3_workspace_status)                         */
+};
+
+/* Human-readable name of a status code (static string, never NULL). */
+EXL3_API const char *exl3_status_string(int status);
+
+/* cudaError_t of the last CUDA failure seen by this thread (0 if none). */
+EXL3_API int exl3_last_cuda_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+EXL3_API int exl3_version(void);
+
+/*
+ * exl3_workspace_bytes -- size of the caller-allocated workspace that
+ * exl3_gemv / exl3_gemm_small_m need for this problem: split-K partial sums
+ * (fp32, L2-resident in practice), one arrival counter per 128-channel output
+ * block and a status word.  The workspace must be zero-filled once before its
+ * first use; every call leaves its counters at zero again, so it can be
+ * reused by later calls on the SAME stream without clearing.  Calls that may
+ * run concurrently need separate workspaces.  Returns 0 for an unsupported
+ * problem.  Host-only, no CUDA call.
+ */
+EXL3_API size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits);
+
+/*
+ * exl3_workspace_status -- synchronises `stream`, then reads and clears the
+ * workspace status word.  Returns EXL3_OK, or EXL3_ERR_TIMEOUT if a kernel
+ * that used this workspace gave up a bounded wait (its output is then not
+ * valid).
+ */
+EXL3_API int exl3_workspace_status(void *workspace, void *stream);
+
+/*
+ * exl3_decode_tiles -- decode a whole trellis-packed matrix to fp16.
+ *   packed : (k_in/16)*(n_out/16)*8*bits uint32 words, tile layout above.
+ *   w_out  : k_in x n_out fp16, row-major (w_out[k*n_out + n] = W[k][n]).
+ *   k_in, n_out : positive multiples of 16.   bits : 2, 3 or 4.
+ * Bit-exact: every output equals the RNE-rounded 3INST weight.
+ */
+EXL3_API int exl3_decode_tiles(const uint32_t *packed, int k_in, int n_out, int bits,
+                      uint16_t *w_out, void *stream);
+
+/*
+ * exl3_hadamard128 -- blockwise normalised Hadamard-128 with a sign vector.
+ *   in, out : rows x n fp16, row-major; out may alias in.
+ *   signs   : n fp16 values, each +1 or -1 (the same vector for every row).
+ *   n       : positive multiple of 128.   rows : >= 1.
+ *   mode 0  : out = H(signs .* in)   (the input-side rotation)
+ *   mode 1  : out = signs .* H(in)   (the output-side rotation)
+ * Computed in fp32, rounded once to fp16 (RNE).
+ */
+EXL3_API int exl3_hadamard128(const uint16_t *in, uint16_t *out, const uint16_t *signs,
+                     int rows, int n, int mode, void *stream);
+
+/*
+ * exl3_gemv -- y = sv .* H(scale .* (H(su .* x) W)) for one input row (M = 1).
+ *   x      : k_in fp16.              packed : trellis words of W (k_in x n_out).
+ *   scale  : n_out fp16.             su : k_in fp16 +-1.   sv : n_out fp16 +-1.
+ *   y      : n_out outputs, fp16 (y_fp32 == 0) or fp32 (y_fp32 != 0).
+ *   k_in, n_out : positive multiples of 128.   bits : 2, 3 or 4.
+ *   workspace, ws_bytes : at least exl3_workspace_bytes(1, k_in, n_out, bits)
+ *                         bytes, zero-filled before first use (see above).
+ * Accumulation is fp32; the reduction order is fixed, so repeated calls give
+ * bitwise-identical y.
+ */
+EXL3_API int exl3_gemv(const uint16_t *x, const uint32_t *packed, const uint16_t *scale,
+              const uint16_t *su, const uint16_t *sv, void *y, int y_fp32,
+              int k_in, int n_out, int bits, void *workspace, size_t ws_bytes,
+              void *stream);
+
+/*
+ * exl3_gemm_small_m -- the same product for m input rows (1 <= m <= 32): the
+ * speculative-draft verification batch.
+ *   x : m x k_in fp16, row-major.   y : m x n_out (fp16 or fp32), row-major.
+ *   Other arguments as exl3_gemv; workspace at least
+ *   exl3_workspace_bytes(m, k_in, n_out, bits).
+ * Deterministic as exl3_gemv.  Different m may use different kernels, which
+ * agree within rounding, not bitwise.
+ */
+EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
+                      const uint16_t *scale, const uint16_t *su, const uint16_t *sv,
+                      void *y, int y_fp32, int k_in, int n_out, int bits,
+                      void *workspace, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXL3_H */

@@ -1,0 +1,103 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every
+entry point include/exl3.h declares, and rejects invalid arguments with the
+documented status codes before touching CUDA.  Only invalid calls are made
+here, so nothing is ever launched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def ex():
+    from gemm_exl3_gemv_b200 import build
+    build.build()
+    from gemm_exl3_gemv_b200 import exl3
+    return exl3
+
+
+def declared_entry_points():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            names += re.findall(r"EXL3_API\s+[\w\s\*]*?\b(exl3_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(ex):
+    names = declared_entry_points()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(ex.lib, n), n
+    assert set(names) == set(ex.EXPORTS)
+
+
+def test_version_and_status_strings(ex):
+    assert ex.lib.exl3_version() >= 100
+    for st in range(8):
+        s = ex.lib.exl3_status_string(st).decode()
+        assert s.startswith("EXL3")
+    assert "unknown" in ex.lib.exl3_status_string(99).decode()
+
+
+def test_workspace_bytes(ex):
+    assert ex.workspace_bytes(1, 5120, 5120, 3) > 0
+    assert ex.workspace_bytes(32, 17408, 5120, 2) >= 32 * 5120 * 4
+    for bad in [(0, 256, 256, 3), (33, 256, 256, 3), (1, 200, 256, 3), (1, 256, 100, 3),
+                (1, 256, 256, 5), (1, 256, 256, 1), (1, -128, 256, 3)]:
+        assert ex.workspace_bytes(*bad) == 0, bad
+
+
+P = ctypes.c_void_p
+
+
+def _gemv(ex, x=16, packed=16, scale=16, su=16, sv=16, y=16, k=256, n=256, bits=3, ws=256, ws_bytes=1 << 20):
+    return ex.lib.exl3_gemv(P(x), P(packed), P(scale), P(su), P(sv), P(y), 0, k, n, bits, P(ws), ws_bytes, None)
+
+
+def test_gemv_argument_validation(ex):
+    assert _gemv(ex, x=0) == ex.EXL3_ERR_INVALID_ARG
+    assert _gemv(ex, y=0) == ex.EXL3_ERR_INVALID_ARG
+    assert _gemv(ex, k=0) == ex.EXL3_ERR_INVALID_ARG
+    assert _gemv(ex, k=200) == ex.EXL3_ERR_UNSUPPORTED
+    assert _gemv(ex, n=136) == ex.EXL3_ERR_UNSUPPORTED
+    assert _gemv(ex, bits=5) == ex.EXL3_ERR_UNSUPPORTED
+    assert _gemv(ex, x=18) == ex.EXL3_ERR_MISALIGNED
+    assert _gemv(ex, packed=20) == ex.EXL3_ERR_MISALIGNED
+    assert _gemv(ex, ws=0) == ex.EXL3_ERR_WORKSPACE
+    assert _gemv(ex, ws_bytes=16) == ex.EXL3_ERR_WORKSPACE
+    assert _gemv(ex, ws=16) == ex.EXL3_ERR_MISALIGNED
+
+
+def test_small_m_validation(ex):
+    f = ex.lib.exl3_gemm_small_m
+    args = lambda m: (m, P(16), P(16), P(16), P(16), P(16), P(16), 0, 256, 256, 3, P(256), 1 << 24, None)
+    assert f(*args(0)) == ex.EXL3_ERR_INVALID_ARG
+    assert f(*args(33)) == ex.EXL3_ERR_UNSUPPORTED
+
+
+def test_decode_and_hadamard_validation(ex):
+    d = ex.lib.exl3_decode_tiles
+    assert d(P(0), 16, 16, 3, P(16), None) == ex.EXL3_ERR_INVALID_ARG
+    assert d(P(16), 24, 16, 3, P(16), None) == ex.EXL3_ERR_UNSUPPORTED
+    assert d(P(16), 16, 16, 6, P(16), None) == ex.EXL3_ERR_UNSUPPORTED
+    assert d(P(16), 16, 16, 3, P(8), None) == ex.EXL3_ERR_MISALIGNED
+    h = ex.lib.exl3_hadamard128
+    assert h(P(16), P(16), P(16), 1, 128, 2, None) == ex.EXL3_ERR_INVALID_ARG
+    assert h(P(16), P(16), P(16), 0, 128, 0, None) == ex.EXL3_ERR_INVALID_ARG
+    assert h(P(16), P(16), P(16), 1, 100, 0, None) == ex.EXL3_ERR_UNSUPPORTED
+    assert h(P(16), P(4), P(16), 1, 128, 0, None) == ex.EXL3_ERR_MISALIGNED
+
+
+def test_product_path_has_no_oracle_or_cpu_fallback():
+    """The binding and the CUDA sources never reference the oracle."""
+    pkg = os.path.join(ROOT, "gemm_exl3_gemv_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")) and f != "synth.py":
+                src = open(os.path.join(dirpath, f)).read()
+                assert "oracle" not in src.lower() or f == "__init__.py", f
