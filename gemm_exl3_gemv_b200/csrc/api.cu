@@ -104,6 +104,12 @@ size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits)
     return exl3::cc_workspace_bytes(m, k_in, n_out, bits);
 }
 
+int exl3_kernel_launches(int m, int k_in, int n_out, int bits)
+{
+    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
+    return exl3::cc_launches(m);
+}
+
 int exl3_workspace_status(void* workspace, void* stream)
 {
     if (!workspace) return EXL3_ERR_INVALID_ARG;

@@ -27,6 +27,7 @@ struct GemmArgs {
 // Split-K factor the CUDA-core kernel uses for this problem (host-only).
 int cc_splits(int m, int k_in, int n_out, int bits);
 size_t cc_workspace_bytes(int m, int k_in, int n_out, int bits);
+int cc_launches(int m);
 cudaError_t launch_gemv_cc(const GemmArgs& a, cudaStream_t stream);
 
 }  // namespace exl3

@@ -20,6 +20,8 @@
 //   * Split-K partial sums go to the workspace; the last CTA of a channel
 //     block (atomic arrival counter) adds them in split order -- fixed, so
 //     results are bitwise repeatable -- scales, rotates and writes y.
+#include <atomic>
+
 #include "exl3_common.cuh"
 #include "exl3_decode.cuh"
 #include "exl3_internal.h"
@@ -300,8 +302,14 @@ cudaError_t launch_t(const GemmArgs& a, int splits, int row0, int rows, cudaStre
     const int krange_max = ((kb_total + splits - 1) / splits) * 128;
     const SmemPlan plan = smem_plan<BITS, MR>(krange_max);
     auto kern = gemv_cc_kernel<BITS, MR>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.total);
-    if (e != cudaSuccess) return e;
+    // raise the dynamic shared-memory limit once per kernel (not per launch, so
+    // launches can be captured in a CUDA graph after the first call)
+    static std::atomic<int> configured{0};
+    if ((int)plan.total > configured.load()) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+        if (e != cudaSuccess) return e;
+        configured.store(200 * 1024);
+    }
     dim3 grid(a.n_out / 128, splits);
     kern<<<grid, kThreads, plan.total, stream>>>(a, splits, krange_max, row0, rows);
     return cudaGetLastError();
@@ -338,6 +346,8 @@ size_t cc_workspace_bytes(int m, int k_in, int n_out, int bits)
     const int s = cc_splits(m, k_in, n_out, bits);
     return ws_part_off(n_out) + (size_t)s * m * n_out * sizeof(float);
 }
+
+int cc_launches(int m) { return (m + 3) / 4; }
 
 cudaError_t launch_gemv_cc(const GemmArgs& a, cudaStream_t stream)
 {

@@ -27,7 +27,7 @@ EXL3_ERR_TIMEOUT = 7
 
 # every entry point include/exl3.h declares
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",
-           "exl3_workspace_status", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
+           "exl3_workspace_status", "exl3_kernel_launches", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
            "exl3_gemm_small_m")
 
 if not os.path.exists(LIB_PATH):
@@ -43,6 +43,8 @@ lib.exl3_version.argtypes = []
 lib.exl3_version.restype = _I
 lib.exl3_workspace_bytes.argtypes = [_I, _I, _I, _I]
 lib.exl3_workspace_bytes.restype = _Z
+lib.exl3_kernel_launches.argtypes = [_I, _I, _I, _I]
+lib.exl3_kernel_launches.restype = _I
 lib.exl3_workspace_status.argtypes = [_P, _P]
 lib.exl3_workspace_status.restype = _I
 lib.exl3_decode_tiles.argtypes = [_P, _I, _I, _I, _P, _P]
@@ -80,6 +82,10 @@ def _stream(stream=None):
 
 def workspace_bytes(m: int, k_in: int, n_out: int, bits: int) -> int:
     return int(lib.exl3_workspace_bytes(m, k_in, n_out, bits))
+
+
+def kernel_launches(m: int, k_in: int, n_out: int, bits: int) -> int:
+    return int(lib.exl3_kernel_launches(m, k_in, n_out, bits))
 
 
 def alloc_workspace(m: int, k_in: int, n_out: int, bits: int, device=None) -> torch.Tensor:

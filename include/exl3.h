@@ -92,6 +92,13 @@ EXL3_API int exl3_version(void);
 EXL3_API size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits);
 
 /*
+ * exl3_kernel_launches -- number of kernel launches one exl3_gemv /
+ * exl3_gemm_small_m call with these arguments enqueues (0 if unsupported).
+ * Host-only, no CUDA call.
+ */
+EXL3_API int exl3_kernel_launches(int m, int k_in, int n_out, int bits);
+
+/*
  * exl3_workspace_status -- synchronises `stream`, then reads and clears the
  * workspace status word.  Returns EXL3_OK, or EXL3_ERR_TIMEOUT if a kernel
  * that used this workspace gave up a bounded wait (its output is then not
