@@ -30,4 +30,10 @@ size_t cc_workspace_bytes(int m, int k_in, int n_out, int bits);
 int cc_launches(int m);
 cudaError_t launch_gemv_cc(const GemmArgs& a, cudaStream_t stream);
 
+// Tensor-core path (2..32 rows): CTA count, workspace size, launcher (two
+// launches per call: input rotation pre-pass and the product kernel).
+int tc_ctas(int m, int k_in, int n_out, int bits);
+size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits);
+cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
+
 }  // namespace exl3
