@@ -6,31 +6,39 @@
 // added on top of upstream", here on B200):
 //     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: m x K_in, y: m x N_out
 //
-// Design:
+// Design (each choice measured on B200):
 //   * A pre-pass writes xt = H(su .* x) once per call, fp16, already laid out
 //     as the MMA's B operand (K-major, 128-byte swizzle), m padded to NT = 16
 //     or 32 rows with zeros.
-//   * Persistent stream-K grid (at most one CTA per SM): the G x TR work units
-//     (128-channel output block g, 16-row tile row tr) are cut into equal
-//     contiguous ranges, one per CTA.  A range may cover the end of one block
-//     and the start of the next; each (CTA, block) piece is a segment.
-//   * Warp roles.  warp 0: 1-D bulk copies of packed tile rows (256*K bytes)
-//     and xt chunks into shared-memory rings.  warp 1: allocates tensor memory
-//     and issues the MMAs (one thread).  warps 2-5: drain the accumulators.
-//     warps 6-13: decode.
+//   * Work unit = one 64-row chunk of K_in for one 128-channel output block
+//     (4 tile rows, 8192 weights).  Persistent stream-K grid: the G x C units
+//     are cut into equal contiguous ranges, at most one CTA per SM.  A range
+//     may cover the end of one block and the start of the next; each
+//     (CTA, block) piece is a segment.
 //   * Decode straight into the A operand: the two fp16 halves of each 3INST
 //     word are kept as two adjacent A rows (lo, hi) of the same input row k,
 //     so the decoded 32-bit word is stored as is and the tensor core adds the
 //     halves.  A is M = 128 rows (64 channels x lo/hi) by K = 16, MN-major with
-//     the 128-byte swizzle; one tile row gives two such MMAs (channels 0-63,
-//     64-127).  The order of the 16 k inside a tile row is permuted (the same
-//     permutation is applied to xt) so that the 16-byte stores of the 32 lanes
-//     are free of bank conflicts.
-//   * Accumulators: two buffers x two channel halves x NT fp32 columns in
-//     tensor memory; a segment's result is drained while the next segment
-//     accumulates.  Segments of a block are combined by the last CTA to finish
-//     (arrival counter) in segment order -- a fixed order, so results are
-//     bitwise repeatable -- which then scales, rotates and writes y.
+//     the 128-byte swizzle; one tile row gives two MMAs (channels 0-63,
+//     64-127).  The 16 k of a tile row are permuted (the same permutation is
+//     applied to xt) so that the 16-byte stores of a warp hit distinct banks.
+//   * 16 decoder warps (4 per scheduler, enough to keep the integer pipes
+//     busy); decoder d always decodes tile row d%4 of every 4th unit into its
+//     own A stage and fetches its own packed words with 1-D bulk copies into a
+//     private 3-slot ring -- bulk-copy issue costs ~85 ns per copy per thread,
+//     so it is spread over 16 threads.
+//   * 4 MMA-issuing threads (one per warp).  A thread that waits on a barrier
+//     right after issuing MMAs stalls until they drain (~0.1 us), so a single
+//     issuer cannot keep the tensor core busy; issuer i takes tile row i of
+//     every unit into its own accumulator, the four interleave on the tensor
+//     core, and the epilogue adds the four accumulators in a fixed order.
+//   * Accumulators in tensor memory: 4 issuers x 2 buffers x 2 channel halves
+//     x NT fp32 columns; a segment is drained while the next accumulates.
+//     Segments of a block are combined by the last CTA to finish (arrival
+//     counter) in segment order -- fixed, so results are bitwise repeatable --
+//     which then scales, rotates and writes y.
+//   * Every wait is bounded (2 s); on expiry the CTA records a timeout in the
+//     workspace status word and winds down.
 #include <atomic>
 #include <utility>
 
@@ -43,31 +51,39 @@ namespace exl3 {
 
 namespace {
 
-constexpr int kDecWarps = 8;
+constexpr int kDecWarps = 16;
+constexpr int kIssuers = 4;
 constexpr int kEpiWarps = 4;
-constexpr int kTcWarps = 2 + kEpiWarps + kDecWarps;
+constexpr int kWarpIss0 = 1;                          // warps 1..4 issue MMAs
+constexpr int kWarpEpi0 = kWarpIss0 + kIssuers;       // warps 5..8 drain accumulators
+constexpr int kWarpDec0 = kWarpEpi0 + kEpiWarps;      // warps 9..24 decode
+constexpr int kTcWarps = kWarpDec0 + kDecWarps;
 constexpr int kTcThreads = 32 * kTcWarps;
-constexpr int kSP = 32;     // packed ring slots (one tile row each)
-constexpr int kSA = 8;      // A stages (one tile row each)
-constexpr int kSB = 4;      // xt stages (one 64-row chunk each)
-constexpr int kABytes = 8192;
+constexpr int kRing = 3;      // packed-word slots per decoder
+constexpr int kSB = 4;        // xt chunk stages
+constexpr int kABytes = 8192; // one tile row of A (128 channels x 16 k x lo/hi x fp16)
 constexpr int kMaxCtas = 148;
-constexpr int kMinUnitsPerCta = 24;
+constexpr int kMinUnitsPerCta = 6;
+constexpr uint32_t kSleepNs = 1000;
+constexpr uint32_t kEpiSleepNs = 10000;
 
 template <int BITS, int NT>
 struct TcLayout {
     static constexpr int ROWB = 256 * BITS;                 // packed bytes per tile row
     static constexpr int BBYTES = NT * 128;                 // xt bytes per 64-row chunk
-    static constexpr int TMEM_COLS = 4 * NT;                // 2 buffers x 2 halves x NT
-    static constexpr int off_a = 0;
-    static constexpr int off_b = off_a + kSA * kABytes;
+    static constexpr int TMEM_COLS = kIssuers * 2 * 2 * NT; // issuers x buffers x halves x NT
+    static constexpr int off_a = 0;                          // kDecWarps A stages
+    static constexpr int off_b = off_a + kDecWarps * kABytes;
     static constexpr int off_p = off_b + kSB * BBYTES;
-    static constexpr int off_z = off_p + kSP * ROWB;
+    static constexpr int off_z = off_p + kDecWarps * kRing * ROWB;
     static constexpr int off_bar = off_z + NT * 128 * 4;
-    static constexpr int nbar = 2 * kSP + 2 * kSA + 2 * kSB + 4;
+    // pfull[dec][ring], afull[dec], aempty[dec], bfull[SB], bempty[SB], dfull[iss][2], dempty[iss][2]
+    static constexpr int nbar = kDecWarps * kRing + 2 * kDecWarps + 2 * kSB + 4 * kIssuers;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
     static_assert(off_b % 1024 == 0 && off_p % 16 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
+    static_assert(TMEM_COLS <= 512, "tensor memory");
+    static_assert(total <= 227 * 1024, "shared memory");
 };
 
 struct TcParams {
@@ -76,8 +92,8 @@ struct TcParams {
     float* part;            // segment partial sums, [slot][NT][128]
     uint32_t* counters;     // per output block
     uint32_t* status;       // workspace status word
-    int G, TR, P;
-    long long U;
+    int G, C, P;            // output blocks, 64-row chunks per block, CTAs
+    long long U;            // units = G * C
 };
 
 __host__ __device__ inline int cta_of_unit(long long x, int P, long long U)
@@ -85,14 +101,17 @@ __host__ __device__ inline int cta_of_unit(long long x, int P, long long U)
     return (int)(((x + 1) * P - 1) / U);
 }
 
-// Bounded wait; also gives up early once another role has aborted.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+// Bounded wait; also gives up early once another role has aborted.  With
+// sleep_ns > 0 the thread may be suspended in hardware between checks.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              uint32_t sleep_ns = 0)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        for (int i = 0; i < 8; ++i) {
+            if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
+        }
         if (*abort_flag) return false;
         if (global_ns() - t0 > 2000000000ull) {
             atomicExch((int*)abort_flag, 1);
@@ -101,16 +120,35 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
+// Warp-wide wait: lane 0 polls, the outcome is broadcast, then every lane
+// observes the completed phase once itself (acquire for each thread).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t sleep_ns = 0)
+{
+    int ok = 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, abort_flag, sleep_ns) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (ok) {
+        // the phase has completed and cannot advance again before this warp
+        // acts on it, so this succeeds at once; bounded all the same
+        int tries = 0;
+        while (!mbar_try_wait(bar, parity) && ++tries < (1 << 20)) {
+        }
+        ok = __all_sync(0xffffffffu, tries < (1 << 20)) ? 1 : 0;
+        if (!ok && (threadIdx.x & 31) == 0) atomicExch((int*)abort_flag, 1);
+    }
+    return ok != 0;
+}
+
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 // Decode the 64 weights of quarter q of tile j (4 input rows x 16 channels)
-// and store the raw 3INST words into the A stage at `ast` (see the layout in
-// the file comment).  soff[rb][t]: per-lane byte offsets of the 16-byte chunk
-// holding channels 4t..4t+3 of a row with (row & 1) == rb; row >> 1 selects
-// the 8-row K group (+2048 bytes).
+// and store the raw 3INST words into the A stage at `ast`.  soff[rb][t]:
+// per-lane byte offset of the 16-byte chunk holding channels 4t..4t+3 of a
+// row with (row & 1) == rb; row >> 1 selects the 8-row K group (+2048 bytes).
 template <int BITS, int NW>
 __device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast, const uint32_t (&soff)[2][4])
 {
@@ -132,18 +170,17 @@ template <int BITS, int NT>
 __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
 {
     using L = TcLayout<BITS, NT>;
-    constexpr int TW = 8 * BITS, QW = 2 * BITS, ROWW = 8 * TW;
+    constexpr int TW = 8 * BITS, QW = 2 * BITS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-    uint64_t* pfull = bar;
-    uint64_t* pempty = pfull + kSP;
-    uint64_t* afull = pempty + kSP;
-    uint64_t* aempty = afull + kSA;
-    uint64_t* bfull = aempty + kSA;
-    uint64_t* bempty = bfull + kSB;
-    uint64_t* dfull = bempty + kSB;
-    uint64_t* dempty = dfull + 2;
+    uint64_t* pfull = bar;                                   // [kDecWarps][kRing]
+    uint64_t* afull = pfull + kDecWarps * kRing;             // [kDecWarps]
+    uint64_t* aempty = afull + kDecWarps;                    // [kDecWarps]
+    uint64_t* bfull = aempty + kDecWarps;                    // [kSB]
+    uint64_t* bempty = bfull + kSB;                          // [kSB]
+    uint64_t* dfull = bempty + kSB;                          // [kIssuers][2]
+    uint64_t* dempty = dfull + 2 * kIssuers;                 // [kIssuers][2]
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort, [2] last-CTA flag
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
@@ -153,20 +190,21 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     const int p = blockIdx.x;
     const long long b0 = (long long)p * prm.U / prm.P;
     const long long b1 = (long long)(p + 1) * prm.U / prm.P;
-    const int n = (int)(b1 - b0);
-    const int TR = prm.TR;
+    const int n = (int)(b1 - b0);                            // units of this CTA
+    const int C = prm.C;
     const int tiles_n = a.n_out / 16;
+    const int g_first = (int)(b0 / C), c_first = (int)(b0 % C);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kSP; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], 1); }
-        for (int i = 0; i < kSA; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
-        for (int i = 0; i < 2; ++i) { mbar_init(&dfull[i], 1); mbar_init(&dempty[i], kEpiWarps); }
+        for (int i = 0; i < kDecWarps * kRing; ++i) mbar_init(&pfull[i], 1);
+        for (int i = 0; i < kDecWarps; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
+        for (int i = 0; i < kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kIssuers); }
+        for (int i = 0; i < 2 * kIssuers; ++i) { mbar_init(&dfull[i], 1); mbar_init(&dempty[i], kEpiWarps); }
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpIss0) {
         tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), L::TMEM_COLS);
         tmem_relinquish();
     }
@@ -176,105 +214,98 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     const uint32_t tmem = (uint32_t)misc[0];
 
     if (warp == 0) {
-        // ------------------------------------------------------ producer ---
+        // ------------------------------------------- xt chunk producer ---
         if (lane == 0) {
-            int bcount = 0;
-            for (int u = 0; u < n; ++u) {
-                const long long unit = b0 + u;
-                const int g = (int)(unit / TR), tr = (int)(unit % TR);
-                if (u == 0 || (tr & 3) == 0) {
-                    const int bs = bcount % kSB;
-                    if (!wait_or_abort(&bempty[bs], ((bcount / kSB) & 1) ^ 1, abort_flag)) break;
-                    mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
-                    bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)(tr >> 2) * L::BBYTES, L::BBYTES,
-                             &bfull[bs]);
-                    ++bcount;
-                }
-                const int s = u % kSP;
-                if (!wait_or_abort(&pempty[s], ((u / kSP) & 1) ^ 1, abort_flag)) break;
-                mbar_arrive_expect_tx(&pfull[s], L::ROWB);
-                bulk_g2s(smem + L::off_p + s * L::ROWB, a.packed + ((size_t)tr * tiles_n + 8 * (size_t)g) * TW,
-                         L::ROWB, &pfull[s]);
+            int c = c_first;
+            for (int u = 0; u < n; ++u, ++c) {
+                if (c == C) c = 0;
+                const int bs = u % kSB;
+                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
+                mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
+                bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)c * L::BBYTES, L::BBYTES, &bfull[bs]);
             }
         }
-    } else if (warp == 1) {
-        // --------------------------------------------------- MMA issuer ---
+    } else if (warp < kWarpEpi0) {
+        // --------------------------------------------------- MMA issuers ---
         if (lane == 0) {
+            const int i = warp - kWarpIss0;               // tile row i of every unit
             constexpr uint32_t idesc = idesc_f16_amn(128, NT);
-            int bcount = 0, seg = 0, cur_b = 0;
-            for (int u = 0; u < n; ++u) {
-                const long long unit = b0 + u;
-                const int tr = (int)(unit % TR);
-                const bool first = (u == 0) || (tr == 0);
-                const bool last = (u == n - 1) || (tr == TR - 1);
-                if (u == 0 || (tr & 3) == 0) {
-                    cur_b = bcount % kSB;
-                    if (!wait_or_abort(&bfull[cur_b], (bcount / kSB) & 1, abort_flag)) break;
-                    ++bcount;
-                }
+            int seg = 0, c = c_first;
+            for (int u = 0; u < n; ++u, ++c) {
+                if (c == C) c = 0;
+                const bool first = (u == 0) || (c == 0);
+                const bool last = (u == n - 1) || (c == C - 1);
+                const int bs = u % kSB;
+                if (!wait_or_abort(&bfull[bs], (u / kSB) & 1, abort_flag)) break;
                 const int db = seg & 1;
-                if (first && !wait_or_abort(&dempty[db], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
-                const int as = u % kSA;
-                if (!wait_or_abort(&afull[as], (u / kSA) & 1, abort_flag)) break;
+                if (first && !wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+                const int st = (u & 3) * 4 + i;            // decoder / A stage of (unit u, row i)
+                if (!wait_or_abort(&afull[st], (u >> 2) & 1, abort_flag)) break;
                 tc_fence_after();
-                const uint32_t abase = smem_u32(smem + L::off_a + as * kABytes);
-                const uint32_t bbase = smem_u32(smem + L::off_b + cur_b * L::BBYTES) + (tr & 3) * 32;
-                const uint64_t bdesc = sdesc_sw128(bbase, 16, 1024);
+                const uint32_t abase = smem_u32(smem + L::off_a + st * kABytes);
+                const uint64_t bdesc = sdesc_sw128(smem_u32(smem + L::off_b + bs * L::BBYTES) + i * 32, 16, 1024);
+                const uint32_t dcol = tmem + (uint32_t)((i * 2 + db) * 2 * NT);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    mma_f16_ss(tmem + db * 2 * NT + h * NT, sdesc_sw128(abase + h * 4096, 1024, 2048), bdesc, idesc,
+                    mma_f16_ss(dcol + h * NT, sdesc_sw128(abase + h * 4096, 1024, 2048), bdesc, idesc,
                                first ? 0u : 1u);
-                mma_commit(&aempty[as]);
-                if ((tr & 3) == 3 || last) mma_commit(&bempty[cur_b]);
+                mma_commit(&aempty[st]);
+                mma_commit(&bempty[bs]);
                 if (last) {
-                    mma_commit(&dfull[db]);
+                    mma_commit(&dfull[2 * i + db]);
                     ++seg;
                 }
             }
         }
-    } else if (warp < 2 + kEpiWarps) {
+    } else if (warp < kWarpDec0) {
         // ----------------------------------------------------- epilogue ---
-        const int ew = warp - 2;            // 0..3
+        const int ew = warp - kWarpEpi0;    // 0..3
         const int quad = warp & 3;          // tensor-memory lanes 32*quad .. 32*quad+31
-        const int et = threadIdx.x - 64;    // 0..127
+        const int et = threadIdx.x - 32 * kWarpEpi0;   // 0..127
         int seg = 0;
-        for (long long u0 = 0; u0 < n; ++seg) {
-            const long long unit = b0 + u0;
-            const int g = (int)(unit / TR), tr0 = (int)(unit % TR);
-            const long long len = (n - u0) < (TR - tr0) ? (n - u0) : (TR - tr0);
-            u0 += len;
+        int u0 = 0, g = g_first, c0 = c_first;
+        while (u0 < n) {
+            const int len = (n - u0) < (C - c0) ? (n - u0) : (C - c0);
             const int db = seg & 1;
-            if (!__all_sync(0xffffffffu, wait_or_abort(&dfull[db], (seg >> 1) & 1, abort_flag))) break;
+            bool ok = true;
+            for (int i = 0; i < kIssuers && ok; ++i)
+                ok = warp_wait(&dfull[2 * i + db], (seg >> 1) & 1, abort_flag, kEpiSleepNs);
+            if (!ok) break;
             tc_fence_after();
-            uint32_t r[2][NT];
+            const int v = 32 * quad + lane;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                float acc[NT];
 #pragma unroll
-                for (int c = 0; c < NT / 16; ++c) {
-                    uint32_t t16[16];
-                    tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + db * 2 * NT + h * NT + 16 * c, t16);
-                    tmem_ld_wait();
+                for (int mm = 0; mm < NT; ++mm) acc[mm] = 0.f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) r[h][16 * c + i] = t16[i];
+                for (int i = 0; i < kIssuers; ++i) {
+#pragma unroll
+                    for (int cc = 0; cc < NT / 16; ++cc) {
+                        uint32_t t16[16];
+                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) +
+                                      (uint32_t)((i * 2 + db) * 2 * NT + h * NT + 16 * cc),
+                                  t16);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) acc[16 * cc + e] += __uint_as_float(t16[e]);
+                    }
+                }
+                // rows 2c (lo) and 2c+1 (hi) of the accumulator belong to channel c
+#pragma unroll
+                for (int mm = 0; mm < NT; ++mm) {
+                    const float sres = acc[mm] + __shfl_xor_sync(0xffffffffu, acc[mm], 1);
+                    if ((lane & 1) == 0) zsm[mm * 128 + 64 * h + (v >> 1)] = sres;
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dempty[db]);
-            // rows 2c (lo) and 2c+1 (hi) of the accumulator belong to channel c
-            const int v = 32 * quad + lane;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-#pragma unroll
-                for (int mm = 0; mm < NT; ++mm) {
-                    float s = __uint_as_float(r[h][mm]);
-                    s += __shfl_xor_sync(0xffffffffu, s, 1);
-                    if ((lane & 1) == 0) zsm[mm * 128 + 64 * h + (v >> 1)] = s;
-                }
-            }
+            if (lane == 0)
+                for (int i = 0; i < kIssuers; ++i) mbar_arrive(&dempty[2 * i + db]);
             named_bar(1, 128);
-            const int p_first = cta_of_unit((long long)g * TR, prm.P, prm.U);
-            const int p_last = cta_of_unit((long long)(g + 1) * TR - 1, prm.P, prm.U);
+            const int p_first = cta_of_unit((long long)g * C, prm.P, prm.U);
+            const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
+            bool finish = true;
             if (p_last > p_first) {
                 float* myslot = prm.part + (size_t)(p + g) * NT * 128;
                 for (int o = et; o < a.m * 128; o += 128) __stcg(myslot + o, zsm[o]);
@@ -285,95 +316,128 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                     misc[2] = (prev == (uint32_t)(p_last - p_first)) ? 1 : 0;
                 }
                 named_bar(1, 128);
-                if (!misc[2]) continue;
-                __threadfence();
-                for (int o = et; o < a.m * 128; o += 128) {
-                    float z = 0.f;
-                    for (int q = p_first; q <= p_last; ++q) z += __ldcg(prm.part + (size_t)(q + g) * NT * 128 + o);
-                    zsm[o] = z;
+                finish = misc[2] != 0;
+                if (finish) {
+                    __threadfence();
+                    for (int o = et; o < a.m * 128; o += 128) {
+                        float z = 0.f;
+                        for (int qq = p_first; qq <= p_last; ++qq)
+                            z += __ldcg(prm.part + (size_t)(qq + g) * NT * 128 + o);
+                        zsm[o] = z;
+                    }
+                    if (et == 0) prm.counters[g] = 0u;
+                    named_bar(1, 128);
                 }
-                if (et == 0) prm.counters[g] = 0u;
-                named_bar(1, 128);
             }
-            // final epilogue for block g: scale, output rotation, signs, store
-            for (int mm = ew; mm < a.m; mm += kEpiWarps) {
-                const int n0 = 128 * g + 4 * lane;
-                const float4 z4 = *reinterpret_cast<const float4*>(zsm + mm * 128 + 4 * lane);
-                const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
-                const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
-                const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
-                const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
-                const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
-                const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
-                float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
-                fwht128_warp(vv);
-                vv[0] *= kInvSqrt128 * sg0.x;
-                vv[1] *= kInvSqrt128 * sg0.y;
-                vv[2] *= kInvSqrt128 * sg1.x;
-                vv[3] *= kInvSqrt128 * sg1.y;
-                const size_t yo = (size_t)mm * a.n_out + n0;
-                if (a.y_fp32) {
-                    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) =
-                        make_float4(vv[0], vv[1], vv[2], vv[3]);
-                } else {
-                    __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
-                    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) = *reinterpret_cast<uint2*>(hh);
+            if (finish) {
+                // final epilogue for block g: scale, output rotation, signs, store
+                for (int mm = ew; mm < a.m; mm += kEpiWarps) {
+                    const int n0 = 128 * g + 4 * lane;
+                    const float4 z4 = *reinterpret_cast<const float4*>(zsm + mm * 128 + 4 * lane);
+                    const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
+                    const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
+                    const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+                    const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+                    const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+                    const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+                    float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
+                    fwht128_warp(vv);
+                    vv[0] *= kInvSqrt128 * sg0.x;
+                    vv[1] *= kInvSqrt128 * sg0.y;
+                    vv[2] *= kInvSqrt128 * sg1.x;
+                    vv[3] *= kInvSqrt128 * sg1.y;
+                    const size_t yo = (size_t)mm * a.n_out + n0;
+                    if (a.y_fp32) {
+                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) =
+                            make_float4(vv[0], vv[1], vv[2], vv[3]);
+                    } else {
+                        __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
+                        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) =
+                            *reinterpret_cast<uint2*>(hh);
+                    }
                 }
             }
             named_bar(1, 128);
+            ++seg;
+            u0 += len;
+            c0 = 0;
+            ++g;
         }
     } else {
         // ------------------------------------------------------ decoders ---
-        const int d = warp - 2 - kEpiWarps;
+        const int d = warp - kWarpDec0;           // 0..15
+        const int slot = d >> 2, t = d & 3;       // units u = slot (mod 4); tile row t of each
         const int j = lane >> 2, q = lane & 3;
         const int src_prev = (lane & ~3) | ((q + 3) & 3);
-        // per-lane store offsets inside an A stage (see decode_quarter_to_a)
         uint32_t soff[2][4];
         {
             const int hh = j >> 2, vgrp = (j >> 1) & 1;
 #pragma unroll
             for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-                for (int t = 0; t < 4; ++t)
-                    soff[rb][t] = hh * 4096 + vgrp * 1024 + (4 * rb + q) * 128 +
-                                  ((uint32_t)(4 * ((j & 1) ^ rb) + (t ^ q)) << 4);
+                for (int tt = 0; tt < 4; ++tt)
+                    soff[rb][tt] = hh * 4096 + vgrp * 1024 + (4 * rb + q) * 128 +
+                                   ((uint32_t)(4 * ((j & 1) ^ rb) + (tt ^ q)) << 4);
         }
-        const uint32_t* pring = reinterpret_cast<const uint32_t*>(smem + L::off_p);
-        const uint32_t abase0 = smem_u32(smem + L::off_a);
-        for (int u = d; u < n; u += kDecWarps) {
-            const int s = u % kSP;
-            if (!__all_sync(0xffffffffu, wait_or_abort(&pfull[s], (u / kSP) & 1, abort_flag))) break;
-            const uint32_t* sw = pring + s * ROWW + j * TW + q * QW;
+        uint8_t* ring = smem + L::off_p + (size_t)d * kRing * L::ROWB;
+        uint64_t* myfull = pfull + d * kRing;
+        const uint32_t ast = smem_u32(smem + L::off_a + d * kABytes);
+        const int nk = n > slot ? (n - slot + 3) / 4 : 0;      // units this decoder handles
+        // packed words of tile row t of the CTA's unit 4k + slot
+        auto src_of = [&](int k) -> const uint32_t* {
+            const long long unit = b0 + 4LL * k + slot;
+            const int g = (int)(unit / C), c = (int)(unit % C);
+            return a.packed + ((size_t)(4 * c + t) * tiles_n + 8 * (size_t)g) * TW;
+        };
+        if (lane == 0) {
+            for (int k = 0; k < kRing && k < nk; ++k) {
+                mbar_arrive_expect_tx(&myfull[k], L::ROWB);
+                bulk_g2s(ring + k * L::ROWB, src_of(k), L::ROWB, &myfull[k]);
+            }
+        }
+        int k = 0;
+        for (; k < nk; ++k) {
+            const int rs = k % kRing;
+            if (!warp_wait(&myfull[rs], (k / kRing) & 1, abort_flag, kSleepNs)) break;
+            const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + rs * L::ROWB) + j * TW + q * QW;
             uint32_t buf[QW + 1];
             if constexpr (QW % 4 == 0) {
 #pragma unroll
-                for (int t = 0; t < QW / 4; ++t) {
-                    const uint4 vv = reinterpret_cast<const uint4*>(sw)[t];
-                    buf[1 + 4 * t] = vv.x; buf[2 + 4 * t] = vv.y; buf[3 + 4 * t] = vv.z; buf[4 + 4 * t] = vv.w;
+                for (int w = 0; w < QW / 4; ++w) {
+                    const uint4 vv = reinterpret_cast<const uint4*>(sw)[w];
+                    buf[1 + 4 * w] = vv.x; buf[2 + 4 * w] = vv.y; buf[3 + 4 * w] = vv.z; buf[4 + 4 * w] = vv.w;
                 }
             } else {
 #pragma unroll
-                for (int t = 0; t < QW / 2; ++t) {
-                    const uint2 vv = reinterpret_cast<const uint2*>(sw)[t];
-                    buf[1 + 2 * t] = vv.x; buf[2 + 2 * t] = vv.y;
+                for (int w = 0; w < QW / 2; ++w) {
+                    const uint2 vv = reinterpret_cast<const uint2*>(sw)[w];
+                    buf[1 + 2 * w] = vv.x; buf[2 + 2 * w] = vv.y;
                 }
             }
             buf[0] = __shfl_sync(0xffffffffu, buf[QW], src_prev);
             __syncwarp();
-            if (lane == 0) mbar_arrive(&pempty[s]);
-            const int as = u % kSA;
-            if (!__all_sync(0xffffffffu, wait_or_abort(&aempty[as], ((u / kSA) & 1) ^ 1, abort_flag))) break;
-            decode_quarter_to_a<BITS>(buf, abase0 + as * kABytes, soff);
+            if (lane == 0 && k + kRing < nk) {
+                fence_proxy_async_smem();
+                mbar_arrive_expect_tx(&myfull[rs], L::ROWB);
+                bulk_g2s(ring + rs * L::ROWB, src_of(k + kRing), L::ROWB, &myfull[rs]);
+            }
+            if (!warp_wait(&aempty[d], (k & 1) ^ 1, abort_flag, kSleepNs)) break;
+            decode_quarter_to_a<BITS>(buf, ast, soff);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[as]);
+            if (lane == 0) mbar_arrive(&afull[d]);
+        }
+        // after an abort, let this warp's copies still in flight land before exit
+        if (k < nk && lane == 0) {
+            for (int kk = k; kk < nk && kk <= k + kRing; ++kk)
+                (void)mbar_wait_bounded(&myfull[kk % kRing], (kk / kRing) & 1, 100000000ull);
         }
     }
 
     // ------------------------------------------------------------ teardown ---
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
+    if (warp == kWarpIss0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -419,8 +483,8 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     TcParams prm;
     prm.a = a;
     prm.G = a.n_out / 128;
-    prm.TR = a.k_in / 16;
-    prm.U = (long long)prm.G * prm.TR;
+    prm.C = a.k_in / 64;
+    prm.U = (long long)prm.G * prm.C;
     prm.P = tc_ctas(a.m, a.k_in, a.n_out, a.bits);
     uint8_t* ws = a.ws;
     prm.status = reinterpret_cast<uint32_t*>(ws);
@@ -452,7 +516,7 @@ int tc_ctas(int m, int k_in, int n_out, int bits)
 {
     (void)m;
     (void)bits;
-    const long long U = (long long)(n_out / 128) * (k_in / 16);
+    const long long U = (long long)(n_out / 128) * (k_in / 64);
     long long p = U / kMinUnitsPerCta;
     if (p > kMaxCtas) p = kMaxCtas;
     if (p < 1) p = 1;
