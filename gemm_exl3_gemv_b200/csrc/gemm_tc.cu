@@ -64,8 +64,8 @@ constexpr int kSB = 4;        // xt chunk stages
 constexpr int kABytes = 8192; // one tile row of A (128 channels x 16 k x lo/hi x fp16)
 constexpr int kMaxCtas = 148;
 constexpr int kMinUnitsPerCta = 6;
-constexpr uint32_t kSleepNs = 1000;
-constexpr uint32_t kEpiSleepNs = 10000;
+constexpr uint32_t kSleepNs = 0;
+constexpr uint32_t kEpiSleepNs = 0;
 
 template <int BITS, int NT>
 struct TcLayout {
@@ -164,6 +164,54 @@ __device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], u
     [&]<int... RT>(std::integer_sequence<int, RT...>) {
         (body(std::integral_constant<int, RT / 4>{}, std::integral_constant<int, RT % 4>{}), ...);
     }(std::make_integer_sequence<int, 16>{});
+}
+
+// zsm[0 .. m*128) = sum of the partial slots (q + g) for q = p_first..p_last,
+// added in that order.  128 threads; each owns up to NT/4 float4 outputs and
+// keeps 2 x NT/4 independent loads in flight (a dependent chain of L2 loads
+// would take ~0.4 us per partial).
+template <int NT>
+__device__ __forceinline__ void reduce_segments(const float* part, int g, int p_first, int p_last, int m, int et,
+                                                float* zsm)
+{
+    constexpr int F = NT / 4;                  // float4 outputs per thread, at most
+    float4 acc[F];
+    const int nf = m * 32;                     // float4 outputs in use
+#pragma unroll
+    for (int r = 0; r < F; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    int qq = p_first;
+    for (; qq + 1 <= p_last; qq += 2) {
+        const float4* s0 = reinterpret_cast<const float4*>(part + (size_t)(qq + g) * NT * 128);
+        const float4* s1 = reinterpret_cast<const float4*>(part + (size_t)(qq + 1 + g) * NT * 128);
+        float4 v0[F], v1[F];
+#pragma unroll
+        for (int r = 0; r < F; ++r) {
+            const int f = et + 128 * r;
+            v0[r] = f < nf ? __ldcg(s0 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v1[r] = f < nf ? __ldcg(s1 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int r = 0; r < F; ++r) {
+            acc[r].x += v0[r].x; acc[r].y += v0[r].y; acc[r].z += v0[r].z; acc[r].w += v0[r].w;
+            acc[r].x += v1[r].x; acc[r].y += v1[r].y; acc[r].z += v1[r].z; acc[r].w += v1[r].w;
+        }
+    }
+    if (qq <= p_last) {
+        const float4* s0 = reinterpret_cast<const float4*>(part + (size_t)(qq + g) * NT * 128);
+#pragma unroll
+        for (int r = 0; r < F; ++r) {
+            const int f = et + 128 * r;
+            if (f < nf) {
+                const float4 v = __ldcg(s0 + f);
+                acc[r].x += v.x; acc[r].y += v.y; acc[r].z += v.z; acc[r].w += v.w;
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < F; ++r) {
+        const int f = et + 128 * r;
+        if (f < nf) reinterpret_cast<float4*>(zsm)[f] = acc[r];
+    }
 }
 
 template <int BITS, int NT>
@@ -307,8 +355,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
             bool finish = true;
             if (p_last > p_first) {
-                float* myslot = prm.part + (size_t)(p + g) * NT * 128;
-                for (int o = et; o < a.m * 128; o += 128) __stcg(myslot + o, zsm[o]);
+                float4* myslot = reinterpret_cast<float4*>(prm.part + (size_t)(p + g) * NT * 128);
+                const float4* z4s = reinterpret_cast<const float4*>(zsm);
+                for (int f = et; f < a.m * 32; f += 128) __stcg(myslot + f, z4s[f]);
                 __threadfence();
                 named_bar(1, 128);
                 if (et == 0) {
@@ -319,12 +368,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                 finish = misc[2] != 0;
                 if (finish) {
                     __threadfence();
-                    for (int o = et; o < a.m * 128; o += 128) {
-                        float z = 0.f;
-                        for (int qq = p_first; qq <= p_last; ++qq)
-                            z += __ldcg(prm.part + (size_t)(qq + g) * NT * 128 + o);
-                        zsm[o] = z;
-                    }
+                    reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, et, zsm);
                     if (et == 0) prm.counters[g] = 0u;
                     named_bar(1, 128);
                 }

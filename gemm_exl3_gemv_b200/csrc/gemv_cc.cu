@@ -244,16 +244,27 @@ __global__ void __launch_bounds__(kThreads, 2)
             return;
         }
         __threadfence();
-        // sum the partials in split order into `red` (as z[mr][n])
+        // sum the partials in split order into `red` (as z[mr][n]); loads are
+        // issued 8 splits at a time so that they are in flight together
 #pragma unroll
         for (int t = 0; t < (MR * 128 + kThreads - 1) / kThreads; ++t) {
             const int o = threadIdx.x + t * kThreads;
             if (o < MR * 128) {
                 const int mr = o / 128, n = o % 128;
                 float z = 0.f;
-                if (mr < rows)
-                    for (int ss = 0; ss < splits; ++ss)
-                        z += __ldcg(part + ((size_t)ss * a.m + row0 + mr) * a.n_out + 128 * g + n);
+                if (mr < rows) {
+                    const float* src = part + ((size_t)row0 + mr) * a.n_out + 128 * g + n;
+                    const size_t stride = (size_t)a.m * a.n_out;
+                    int ss = 0;
+                    for (; ss + 8 <= splits; ss += 8) {
+                        float v[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[e] = __ldcg(src + (size_t)(ss + e) * stride);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) z += v[e];
+                    }
+                    for (; ss < splits; ++ss) z += __ldcg(src + (size_t)ss * stride);
+                }
                 red[o] = z;
             }
         }
