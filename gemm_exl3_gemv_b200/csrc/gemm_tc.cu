@@ -23,15 +23,16 @@
 //     64-127).  The 16 k of a tile row are permuted (the same permutation is
 //     applied to xt) so that the 16-byte stores of a warp hit distinct banks.
 //   * 16 decoder warps (4 per scheduler, enough to keep the integer pipes
-//     busy); decoder d always decodes tile row d%4 of every 4th unit into its
-//     own A stage and fetches its own packed words with 1-D bulk copies into a
+//     busy); decoder d always decodes tile row d%4 of the units u = d/4
+//     (mod 4) into its own A stage and fetches its own packed words with 1-D bulk copies into a
 //     private 3-slot ring -- bulk-copy issue costs ~85 ns per copy per thread,
 //     so it is spread over 16 threads.
 //   * 4 MMA-issuing threads (one per warp).  A thread that waits on a barrier
 //     right after issuing MMAs stalls until they drain (~0.1 us), so a single
-//     issuer cannot keep the tensor core busy; issuer i takes tile row i of
-//     every unit into its own accumulator, the four interleave on the tensor
-//     core, and the epilogue adds the four accumulators in a fixed order.
+//     issuer cannot keep the tensor core busy; issuer i takes every unit
+//     u = i (mod 4) (8 MMAs per barrier wait) into its own accumulator, the
+//     four interleave on the tensor core, and the epilogue adds the four
+//     accumulators in a fixed order.
 //   * Accumulators in tensor memory: 4 issuers x 2 buffers x 2 channel halves
 //     x NT fp32 columns; a segment is drained while the next accumulates.
 //     Segments of a block are combined by the last CTA to finish (arrival
@@ -60,10 +61,11 @@ constexpr int kWarpDec0 = kWarpEpi0 + kEpiWarps;      // warps 9..24 decode
 constexpr int kTcWarps = kWarpDec0 + kDecWarps;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kRing = 3;      // packed-word slots per decoder
-constexpr int kSB = 4;        // xt chunk stages
-constexpr int kABytes = 8192; // one tile row of A (128 channels x 16 k x lo/hi x fp16)
+constexpr int kSB = 6;        // xt chunk stages
+constexpr int kABytes = 4096; // one tile row of A (128 channels x 16 k, fp16)
+constexpr int kABuf = 2;      // A stages per decoder (double buffered)
 constexpr int kMaxCtas = 148;
-constexpr int kMinUnitsPerCta = 6;
+constexpr int kMinUnitsPerCta = 10;
 constexpr uint32_t kSleepNs = 0;
 constexpr uint32_t kEpiSleepNs = 0;
 
@@ -71,18 +73,18 @@ template <int BITS, int NT>
 struct TcLayout {
     static constexpr int ROWB = 256 * BITS;                 // packed bytes per tile row
     static constexpr int BBYTES = NT * 128;                 // xt bytes per 64-row chunk
-    static constexpr int TMEM_COLS = kIssuers * 2 * 2 * NT; // issuers x buffers x halves x NT
-    static constexpr int off_a = 0;                          // kDecWarps A stages
-    static constexpr int off_b = off_a + kDecWarps * kABytes;
+    static constexpr int TMEM_COLS = kIssuers * 2 * NT;     // issuers x buffers x NT columns
+    static constexpr int off_a = 0;                          // kABuf x kDecWarps A stages
+    static constexpr int off_b = off_a + kABuf * kDecWarps * kABytes;
     static constexpr int off_p = off_b + kSB * BBYTES;
     static constexpr int off_z = off_p + kDecWarps * kRing * ROWB;
     static constexpr int off_bar = off_z + NT * 128 * 4;
-    // pfull[dec][ring], afull[dec], aempty[dec], bfull[SB], bempty[SB], dfull[iss][2], dempty[iss][2]
-    static constexpr int nbar = kDecWarps * kRing + 2 * kDecWarps + 2 * kSB + 4 * kIssuers;
+    // pfull[dec][ring], afull[slot][buf], aempty[slot][buf], bfull[SB], bempty[SB], dfull[iss][2], dempty[iss][2]
+    static constexpr int nbar = kDecWarps * kRing + 2 * kIssuers * kABuf + 2 * kSB + 4 * kIssuers;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
     static_assert(off_b % 1024 == 0 && off_p % 16 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
-    static_assert(TMEM_COLS <= 512, "tensor memory");
+    static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512, "tensor memory");
     static_assert(total <= 227 * 1024, "shared memory");
 };
 
@@ -146,24 +148,44 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, ui
 }
 
 // Decode the 64 weights of quarter q of tile j (4 input rows x 16 channels)
-// and store the raw 3INST words into the A stage at `ast`.  soff[rb][t]:
-// per-lane byte offset of the 16-byte chunk holding channels 4t..4t+3 of a
-// row with (row & 1) == rb; row >> 1 selects the 8-row K group (+2048 bytes).
+// into fp16 (the two halves of each 3INST word added and rounded once, RNE:
+// the exact decoded weight) and store them into the A stage at `ast`, two
+// 16-byte chunks per row.  soff[rb][e]: per-lane byte offset of the chunk
+// holding channels 8e..8e+7 of a row with (row & 1) == rb; row >> 1 selects
+// the 8-row K group (+2048 bytes).
 template <int BITS, int NW>
-__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast, const uint32_t (&soff)[2][4])
+__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast, const uint32_t (&soff)[2][2])
 {
-    // fully unrolled over (row r, chunk t): every window position is a compile-time constant
-    auto body = [&](auto R, auto T) {
-        constexpr int r = decltype(R)::value, t = decltype(T)::value;
-        const uint32_t m0 = inst3(window16<(16 * r + 4 * t + 1) * BITS + 16>(buf));
-        const uint32_t m1 = inst3(window16<(16 * r + 4 * t + 2) * BITS + 16>(buf));
-        const uint32_t m2 = inst3(window16<(16 * r + 4 * t + 3) * BITS + 16>(buf));
-        const uint32_t m3 = inst3(window16<(16 * r + 4 * t + 4) * BITS + 16>(buf));
-        sts128(ast + soff[r & 1][t] + (r >> 1) * 2048, m0, m1, m2, m3);
+    // fully unrolled over (row r, chunk e): every window position is a compile-time constant
+    auto body = [&](auto R, auto E) {
+        constexpr int r = decltype(R)::value, e = decltype(E)::value;
+        // channels 8e + 2c, 8e + 2c + 1 of row r -> one fp16 pair
+        auto pair = [&](auto Cc) -> uint32_t {
+            constexpr int c = decltype(Cc)::value;
+            const __half a = weight_of(inst3(window16<(16 * r + 8 * e + 2 * c + 1) * BITS + 16>(buf)));
+            const __half b = weight_of(inst3(window16<(16 * r + 8 * e + 2 * c + 2) * BITS + 16>(buf)));
+            __half2 h = __halves2half2(a, b);
+            return *reinterpret_cast<uint32_t*>(&h);
+        };
+        sts128(ast + soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
+               pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
+               pair(std::integral_constant<int, 3>{}));
     };
-    [&]<int... RT>(std::integer_sequence<int, RT...>) {
-        (body(std::integral_constant<int, RT / 4>{}, std::integral_constant<int, RT % 4>{}), ...);
-    }(std::make_integer_sequence<int, 16>{});
+    [&]<int... RE>(std::integer_sequence<int, RE...>) {
+        (body(std::integral_constant<int, RE / 2>{}, std::integral_constant<int, RE % 2>{}), ...);
+    }(std::make_integer_sequence<int, 8>{});
+}
+
+// Row v of an accumulator (row v of A) holds output channel chan_of_row(v):
+// tile j's 16 channels fill 16-byte chunks 4*(j&1) + 2*((j>>1)&1) + e of MN
+// atom j/4 (e = channel/8), so that the 8 lanes of a store phase hit 8
+// different banks.
+__host__ __device__ constexpr int chunk_of_tile(int j4, int e) { return 4 * (j4 & 1) + 2 * ((j4 >> 1) & 1) + e; }
+__device__ __forceinline__ int chan_of_row(int v)
+{
+    const int atom = v >> 6, chunk = (v >> 3) & 7, pos = v & 7;
+    const int j4 = 2 * ((chunk >> 1) & 1) + ((chunk >> 2) & 1);
+    return 16 * (4 * atom + j4) + 8 * (chunk & 1) + pos;
 }
 
 // zsm[0 .. m*128) = sum of the partial slots (q + g) for q = p_first..p_last,
@@ -223,9 +245,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
     uint64_t* pfull = bar;                                   // [kDecWarps][kRing]
-    uint64_t* afull = pfull + kDecWarps * kRing;             // [kDecWarps]
-    uint64_t* aempty = afull + kDecWarps;                    // [kDecWarps]
-    uint64_t* bfull = aempty + kDecWarps;                    // [kSB]
+    uint64_t* afull = pfull + kDecWarps * kRing;             // [slot][buf]: the 4 decoders of a slot arrive
+    uint64_t* aempty = afull + kIssuers * kABuf;             // [slot][buf]: the slot's issuer commits
+    uint64_t* bfull = aempty + kIssuers * kABuf;             // [kSB]
     uint64_t* bempty = bfull + kSB;                          // [kSB]
     uint64_t* dfull = bempty + kSB;                          // [kIssuers][2]
     uint64_t* dempty = dfull + 2 * kIssuers;                 // [kIssuers][2]
@@ -245,8 +267,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDecWarps * kRing; ++i) mbar_init(&pfull[i], 1);
-        for (int i = 0; i < kDecWarps; ++i) { mbar_init(&afull[i], 1); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kIssuers); }
+        for (int i = 0; i < kIssuers * kABuf; ++i) { mbar_init(&afull[i], 4); mbar_init(&aempty[i], 1); }
+        for (int i = 0; i < kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
         for (int i = 0; i < 2 * kIssuers; ++i) { mbar_init(&dfull[i], 1); mbar_init(&dempty[i], kEpiWarps); }
         misc[1] = 0;
         misc[2] = 0;
@@ -268,41 +290,48 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             for (int u = 0; u < n; ++u, ++c) {
                 if (c == C) c = 0;
                 const int bs = u % kSB;
-                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
+                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag)) break;
                 mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
                 bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)c * L::BBYTES, L::BBYTES, &bfull[bs]);
             }
         }
     } else if (warp < kWarpEpi0) {
         // --------------------------------------------------- MMA issuers ---
+        // Issuer i takes the units u = i (mod 4) -- all 4 tile rows, 8 MMAs per
+        // barrier wait -- into its own accumulator.  It takes part in every
+        // segment (waits for its buffer, commits it) even when it has no unit
+        // there, so that every barrier sees one phase per segment.
         if (lane == 0) {
-            const int i = warp - kWarpIss0;               // tile row i of every unit
+            const int i = warp - kWarpIss0;
             constexpr uint32_t idesc = idesc_f16_amn(128, NT);
-            int seg = 0, c = c_first;
-            for (int u = 0; u < n; ++u, ++c) {
-                if (c == C) c = 0;
-                const bool first = (u == 0) || (c == 0);
-                const bool last = (u == n - 1) || (c == C - 1);
-                const int bs = u % kSB;
-                if (!wait_or_abort(&bfull[bs], (u / kSB) & 1, abort_flag)) break;
+            int seg = 0, u0 = 0, c0 = c_first;
+            bool ok = true;
+            while (ok && u0 < n) {
+                const int len = (n - u0) < (C - c0) ? (n - u0) : (C - c0);
                 const int db = seg & 1;
-                if (first && !wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
-                const int st = (u & 3) * 4 + i;            // decoder / A stage of (unit u, row i)
-                if (!wait_or_abort(&afull[st], (u >> 2) & 1, abort_flag)) break;
-                tc_fence_after();
-                const uint32_t abase = smem_u32(smem + L::off_a + st * kABytes);
-                const uint64_t bdesc = sdesc_sw128(smem_u32(smem + L::off_b + bs * L::BBYTES) + i * 32, 16, 1024);
-                const uint32_t dcol = tmem + (uint32_t)((i * 2 + db) * 2 * NT);
+                if (!wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+                const uint32_t dcol = tmem + (uint32_t)((i * 2 + db) * NT);
+                bool first = true;
+                for (int u = u0 + ((i - u0) & 3); u < u0 + len; u += 4) {
+                    const int k = u >> 2, ab = k & 1;            // k-th unit of slot i, A buffer
+                    if (!wait_or_abort(&afull[i * kABuf + ab], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const int bs = u % kSB;
+                    const uint32_t bbase = smem_u32(smem + L::off_b + bs * L::BBYTES);
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    mma_f16_ss(dcol + h * NT, sdesc_sw128(abase + h * 4096, 1024, 2048), bdesc, idesc,
-                               first ? 0u : 1u);
-                mma_commit(&aempty[st]);
-                mma_commit(&bempty[bs]);
-                if (last) {
-                    mma_commit(&dfull[2 * i + db]);
-                    ++seg;
+                    for (int t = 0; t < 4; ++t) {
+                        const uint32_t abase = smem_u32(smem + L::off_a + (ab * kDecWarps + i * 4 + t) * kABytes);
+                        mma_f16_ss(dcol, sdesc_sw128(abase, 1024, 2048), sdesc_sw128(bbase + t * 32, 16, 1024), idesc,
+                                   (first && t == 0) ? 0u : 1u);
+                    }
+                    first = false;
+                    mma_commit(&aempty[i * kABuf + ab]);
+                    mma_commit(&bempty[bs]);
                 }
+                mma_commit(&dfull[2 * i + db]);
+                ++seg;
+                u0 += len;
+                c0 = 0;
             }
         }
     } else if (warp < kWarpDec0) {
@@ -320,31 +349,26 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                 ok = warp_wait(&dfull[2 * i + db], (seg >> 1) & 1, abort_flag, kEpiSleepNs);
             if (!ok) break;
             tc_fence_after();
-            const int v = 32 * quad + lane;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            {
+                const int v = 32 * quad + lane;
                 float acc[NT];
 #pragma unroll
                 for (int mm = 0; mm < NT; ++mm) acc[mm] = 0.f;
 #pragma unroll
                 for (int i = 0; i < kIssuers; ++i) {
+                    if (len < 4 && ((i - u0) & 3) >= len) continue;   // issuer i had no unit here
 #pragma unroll
                     for (int cc = 0; cc < NT / 16; ++cc) {
                         uint32_t t16[16];
-                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) +
-                                      (uint32_t)((i * 2 + db) * 2 * NT + h * NT + 16 * cc),
-                                  t16);
+                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((i * 2 + db) * NT + 16 * cc), t16);
                         tmem_ld_wait();
 #pragma unroll
                         for (int e = 0; e < 16; ++e) acc[16 * cc + e] += __uint_as_float(t16[e]);
                     }
                 }
-                // rows 2c (lo) and 2c+1 (hi) of the accumulator belong to channel c
+                const int ch = chan_of_row(v);
 #pragma unroll
-                for (int mm = 0; mm < NT; ++mm) {
-                    const float sres = acc[mm] + __shfl_xor_sync(0xffffffffu, acc[mm], 1);
-                    if ((lane & 1) == 0) zsm[mm * 128 + 64 * h + (v >> 1)] = sres;
-                }
+                for (int mm = 0; mm < NT; ++mm) zsm[mm * 128 + ch] = acc[mm];
             }
             tc_fence_before();
             __syncwarp();
@@ -413,19 +437,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
         const int slot = d >> 2, t = d & 3;       // units u = slot (mod 4); tile row t of each
         const int j = lane >> 2, q = lane & 3;
         const int src_prev = (lane & ~3) | ((q + 3) & 3);
-        uint32_t soff[2][4];
+        uint32_t soff[2][2];
         {
-            const int hh = j >> 2, vgrp = (j >> 1) & 1;
+            const int atom = j >> 2, j4 = j & 3;
 #pragma unroll
             for (int rb = 0; rb < 2; ++rb)
 #pragma unroll
-                for (int tt = 0; tt < 4; ++tt)
-                    soff[rb][tt] = hh * 4096 + vgrp * 1024 + (4 * rb + q) * 128 +
-                                   ((uint32_t)(4 * ((j & 1) ^ rb) + (tt ^ q)) << 4);
+                for (int e = 0; e < 2; ++e)
+                    soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
         }
         uint8_t* ring = smem + L::off_p + (size_t)d * kRing * L::ROWB;
         uint64_t* myfull = pfull + d * kRing;
-        const uint32_t ast = smem_u32(smem + L::off_a + d * kABytes);
+        const uint32_t ast0 = smem_u32(smem + L::off_a + d * kABytes);  // stage d (+ kDecWarps for buffer 1)
         const int nk = n > slot ? (n - slot + 3) / 4 : 0;      // units this decoder handles
         // packed words of tile row t of the CTA's unit 4k + slot
         auto src_of = [&](int k) -> const uint32_t* {
@@ -465,11 +488,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                 mbar_arrive_expect_tx(&myfull[rs], L::ROWB);
                 bulk_g2s(ring + rs * L::ROWB, src_of(k + kRing), L::ROWB, &myfull[rs]);
             }
-            if (!warp_wait(&aempty[d], (k & 1) ^ 1, abort_flag, kSleepNs)) break;
-            decode_quarter_to_a<BITS>(buf, ast, soff);
+            const int ab = k & 1;
+            if (!warp_wait(&aempty[slot * kABuf + ab], ((k >> 1) & 1) ^ 1, abort_flag, kSleepNs)) break;
+            decode_quarter_to_a<BITS>(buf, ast0 + ab * kDecWarps * kABytes, soff);
             fence_proxy_async_smem();
+            // the unit's xt chunk must have landed before its MMAs are issued;
+            // the decoder checks it here so that the issuers wait only on afull
+            const int ub = 4 * k + slot;
+            if (!warp_wait(&bfull[ub % kSB], (ub / kSB) & 1, abort_flag)) break;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[d]);
+            if (lane == 0) mbar_arrive(&afull[slot * kABuf + ab]);
         }
         // after an abort, let this warp's copies still in flight land before exit
         if (k < nk && lane == 0) {
