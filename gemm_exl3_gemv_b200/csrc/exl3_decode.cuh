@@ -48,4 +48,16 @@ __device__ __forceinline__ __half weight_of(uint32_t m)
     return __hadd(__low2half(h), __high2half(h));
 }
 
+// Two decoded weights packed as fp16 (w(ma) in the low half, w(mb) in the
+// high half): the low halves and the high halves of the two 3INST words are
+// gathered with byte permutes and added in one packed fp16 add (RNE), which
+// gives the same bits as weight_of on each word.
+__device__ __forceinline__ uint32_t weight_pair(uint32_t ma, uint32_t mb)
+{
+    const uint32_t lo = __byte_perm(ma, mb, 0x5410);   // (ma[15:0], mb[15:0])
+    const uint32_t hi = __byte_perm(ma, mb, 0x7632);   // (ma[31:16], mb[31:16])
+    __half2 s = __hadd2(*reinterpret_cast<const __half2*>(&lo), *reinterpret_cast<const __half2*>(&hi));
+    return *reinterpret_cast<uint32_t*>(&s);
+}
+
 }  // namespace exl3

@@ -66,8 +66,11 @@ constexpr int kABytes = 4096; // one tile row of A (128 channels x 16 k, fp16)
 constexpr int kABuf = 2;      // A stages per decoder (double buffered)
 constexpr int kMaxCtas = 148;
 constexpr int kMinUnitsPerCta = 10;
-constexpr uint32_t kSleepNs = 0;
-constexpr uint32_t kEpiSleepNs = 0;
+// Suspend hints for barrier waits (ns): waiting threads are parked in
+// hardware instead of polling, leaving the issue slots to the decoders.
+constexpr uint32_t kSleepNs = 2000;
+constexpr uint32_t kIssSleepNs = 1000;
+constexpr uint32_t kEpiSleepNs = 20000;
 
 template <int BITS, int NT>
 struct TcLayout {
@@ -104,7 +107,8 @@ __host__ __device__ inline int cta_of_unit(long long x, int P, long long U)
 }
 
 // Bounded wait; also gives up early once another role has aborted.  With
-// sleep_ns > 0 the thread may be suspended in hardware between checks.
+// sleep_ns > 0 the thread may be suspended in hardware between checks (it is
+// resumed when the phase completes).
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                               uint32_t sleep_ns = 0)
 {
@@ -162,10 +166,9 @@ __device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], u
         // channels 8e + 2c, 8e + 2c + 1 of row r -> one fp16 pair
         auto pair = [&](auto Cc) -> uint32_t {
             constexpr int c = decltype(Cc)::value;
-            const __half a = weight_of(inst3(window16<(16 * r + 8 * e + 2 * c + 1) * BITS + 16>(buf)));
-            const __half b = weight_of(inst3(window16<(16 * r + 8 * e + 2 * c + 2) * BITS + 16>(buf)));
-            __half2 h = __halves2half2(a, b);
-            return *reinterpret_cast<uint32_t*>(&h);
+            const uint32_t ma = inst3(window16<(16 * r + 8 * e + 2 * c + 1) * BITS + 16>(buf));
+            const uint32_t mb = inst3(window16<(16 * r + 8 * e + 2 * c + 2) * BITS + 16>(buf));
+            return weight_pair(ma, mb);
         };
         sts128(ast + soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
                pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             for (int u = 0; u < n; ++u, ++c) {
                 if (c == C) c = 0;
                 const int bs = u % kSB;
-                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag)) break;
+                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
                 mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
                 bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)c * L::BBYTES, L::BBYTES, &bfull[bs]);
             }
@@ -309,12 +312,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             while (ok && u0 < n) {
                 const int len = (n - u0) < (C - c0) ? (n - u0) : (C - c0);
                 const int db = seg & 1;
-                if (!wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag)) break;
+                if (!wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag, kIssSleepNs)) break;
                 const uint32_t dcol = tmem + (uint32_t)((i * 2 + db) * NT);
                 bool first = true;
                 for (int u = u0 + ((i - u0) & 3); u < u0 + len; u += 4) {
                     const int k = u >> 2, ab = k & 1;            // k-th unit of slot i, A buffer
-                    if (!wait_or_abort(&afull[i * kABuf + ab], (k >> 1) & 1, abort_flag)) { ok = false; break; }
+                    if (!wait_or_abort(&afull[i * kABuf + ab], (k >> 1) & 1, abort_flag, kIssSleepNs)) { ok = false; break; }
                     tc_fence_after();
                     const int bs = u % kSB;
                     const uint32_t bbase = smem_u32(smem + L::off_b + bs * L::BBYTES);
@@ -450,16 +453,20 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
         uint64_t* myfull = pfull + d * kRing;
         const uint32_t ast0 = smem_u32(smem + L::off_a + d * kABytes);  // stage d (+ kDecWarps for buffer 1)
         const int nk = n > slot ? (n - slot + 3) / 4 : 0;      // units this decoder handles
-        // packed words of tile row t of the CTA's unit 4k + slot
-        auto src_of = [&](int k) -> const uint32_t* {
-            const long long unit = b0 + 4LL * k + slot;
-            const int g = (int)(unit / C), c = (int)(unit % C);
-            return a.packed + ((size_t)(4 * c + t) * tiles_n + 8 * (size_t)g) * TW;
+        // (block, chunk) of the next unit to prefetch, walked by steps of 4
+        // units (no division per unit)
+        int pf_g = g_first, pf_c = c_first + slot;
+        while (pf_c >= C) { pf_c -= C; ++pf_g; }
+        auto next_src = [&]() -> const uint32_t* {
+            const uint32_t* src = a.packed + ((size_t)(4 * pf_c + t) * tiles_n + 8 * (size_t)pf_g) * TW;
+            pf_c += 4;
+            while (pf_c >= C) { pf_c -= C; ++pf_g; }
+            return src;
         };
         if (lane == 0) {
             for (int k = 0; k < kRing && k < nk; ++k) {
                 mbar_arrive_expect_tx(&myfull[k], L::ROWB);
-                bulk_g2s(ring + k * L::ROWB, src_of(k), L::ROWB, &myfull[k]);
+                bulk_g2s(ring + k * L::ROWB, next_src(), L::ROWB, &myfull[k]);
             }
         }
         int k = 0;
@@ -486,7 +493,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             if (lane == 0 && k + kRing < nk) {
                 fence_proxy_async_smem();
                 mbar_arrive_expect_tx(&myfull[rs], L::ROWB);
-                bulk_g2s(ring + rs * L::ROWB, src_of(k + kRing), L::ROWB, &myfull[rs]);
+                bulk_g2s(ring + rs * L::ROWB, next_src(), L::ROWB, &myfull[rs]);
             }
             const int ab = k & 1;
             if (!warp_wait(&aempty[slot * kABuf + ab], ((k >> 1) & 1) ^ 1, abort_flag, kSleepNs)) break;
@@ -495,7 +502,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             // the unit's xt chunk must have landed before its MMAs are issued;
             // the decoder checks it here so that the issuers wait only on afull
             const int ub = 4 * k + slot;
-            if (!warp_wait(&bfull[ub % kSB], (ub / kSB) & 1, abort_flag)) break;
+            if (!warp_wait(&bfull[ub % kSB], (ub / kSB) & 1, abort_flag, kSleepNs)) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[slot * kABuf + ab]);
         }
