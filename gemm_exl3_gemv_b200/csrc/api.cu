@@ -2,6 +2,7 @@
 // argument validation on the host, architecture check, dispatch to kernels.
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "../../include/exl3.h"
 #include "exl3_common.cuh"
@@ -166,3 +167,82 @@ int exl3_gemm_small_m(int m, const uint16_t* x, const uint32_t* packed, const ui
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------ no-allocation GEMV ---
+//
+// exl3_gemv_noalloc: the single-row product without a caller workspace, for
+// callers that cannot allocate device memory (see include/exl3.h).  Its
+// split-K scratch is this file-scope device array.  In host code the name
+// g_noalloc_scratch is only a host-side stand-in, so its device address is
+// looked up once per device (cudaGetSymbolAddress, with that device current)
+// and passed to the kernel as the workspace pointer.
+
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;   // held by every device that loads the library
+
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device).
+int noalloc_scratch(void** out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return EXL3_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e);
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return EXL3_OK;
+}
+
+}  // namespace
+
+extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, const uint16_t* scale,
+                                 const uint16_t* su, const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out,
+                                 int bits, void* stream)
+{
+    if (!x || !packed || !scale || !su || !sv || !y) return EXL3_ERR_INVALID_ARG;
+    if (k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
+    if (!bits_ok(bits) || k_in % 128 || n_out % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(su) || !aligned16(sv) ||
+        !aligned16(y))
+        return EXL3_ERR_MISALIGNED;
+    const size_t need = exl3_workspace_bytes(1, k_in, n_out, bits);
+    if (need == 0 || need > kNoAllocScratchBytes) return EXL3_ERR_WORKSPACE;   // beyond the fixed scratch
+    int st = check_arch();
+    if (st != EXL3_OK) return st;
+    void* ws = nullptr;
+    st = noalloc_scratch(&ws);
+    if (st != EXL3_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // the array keeps the last call's contents: the status word and the
+    // arrival counters must start at zero
+    cudaError_t e = cudaMemsetAsync(ws, 0, exl3::ws_part_off(n_out), s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    exl3::GemmArgs a;
+    a.x = x;
+    a.packed = packed;
+    a.scale = scale;
+    a.su = su;
+    a.sv = sv;
+    a.y = y;
+    a.y_fp32 = y_fp32 ? 1 : 0;
+    a.m = 1;
+    a.k_in = k_in;
+    a.n_out = n_out;
+    a.bits = bits;
+    a.ws = static_cast<unsigned char*>(ws);
+    e = exl3::launch_gemv_cc(a, s);
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}

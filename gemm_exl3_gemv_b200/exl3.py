@@ -28,7 +28,7 @@ EXL3_ERR_TIMEOUT = 7
 # every entry point include/exl3.h declares
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",
            "exl3_workspace_status", "exl3_kernel_launches", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
-           "exl3_gemm_small_m")
+           "exl3_gemm_small_m", "exl3_gemv_noalloc")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libexl3.so not built ({LIB_PATH}); run `python -m gemm_exl3_gemv_b200.build`")
@@ -55,6 +55,8 @@ lib.exl3_gemv.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]
 lib.exl3_gemv.restype = _I
 lib.exl3_gemm_small_m.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]
 lib.exl3_gemm_small_m.restype = _I
+lib.exl3_gemv_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+lib.exl3_gemv_noalloc.restype = _I
 
 
 class Exl3Error(RuntimeError):

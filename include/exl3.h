@@ -158,6 +158,33 @@ EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
                       void *y, int y_fp32, int k_in, int n_out, int bits,
                       void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * exl3_gemv_noalloc -- exl3_gemv without a workspace argument.  The paper has
+ * no counterpart of this entry point; it exists for callers that cannot
+ * allocate device memory on the call path -- for example an inference engine
+ * that reserves all of HBM for its own pool at start-up and forbids further
+ * cudaMalloc, or a plugin whose host application owns the CUDA allocator --
+ * and therefore cannot hand in the split-K workspace exl3_gemv needs.
+ *   Arguments: as exl3_gemv, minus workspace and ws_bytes.
+ *   Scratch: a fixed device array of 4 MiB inside the library, which every
+ *     GPU that loads the library holds until the process exits.  Problems whose
+ *     workspace (exl3_workspace_bytes(1, k_in, n_out, bits)) exceeds it are
+ *     rejected with EXL3_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   Allocation: none -- no cudaMalloc, cudaFree or allocating library call.
+ *     Each call clears the array's counters with cudaMemsetAsync on `stream`.
+ *   Concurrency: all calls on a device share the one array, so calls that
+ *     may overlap on the GPU (different streams without ordering) race and
+ *     give wrong results; serialise them, or use exl3_gemv with separate
+ *     workspaces.
+ * Results are the same as exl3_gemv's.
+ */
+EXL3_API int exl3_gemv_noalloc(const uint16_t *x, const uint32_t *packed, const uint16_t *scale,
+                               const uint16_t *su, const uint16_t *sv, void *y, int y_fp32,
+                               int k_in, int n_out, int bits, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
