@@ -55,13 +55,14 @@ namespace {
 constexpr int kDecWarps = 16;
 constexpr int kIssuers = 4;
 constexpr int kEpiWarps = 4;
-constexpr int kWarpIss0 = 1;                          // warps 1..4 issue MMAs
-constexpr int kWarpEpi0 = kWarpIss0 + kIssuers;       // warps 5..8 drain accumulators
-constexpr int kWarpDec0 = kWarpEpi0 + kEpiWarps;      // warps 9..24 decode
+constexpr int kWarpProd0 = 0;                         // warps 0..3 issue the bulk copies of slots 0..3
+constexpr int kWarpIss0 = 4;                          // warps 4..7 issue MMAs
+constexpr int kWarpEpi0 = kWarpIss0 + kIssuers;       // warps 8..11 drain accumulators
+constexpr int kWarpDec0 = kWarpEpi0 + kEpiWarps;      // warps 12..27 decode
 constexpr int kTcWarps = kWarpDec0 + kDecWarps;
 constexpr int kTcThreads = 32 * kTcWarps;
 constexpr int kRing = 3;      // packed-word slots per decoder
-constexpr int kSB = 6;        // xt chunk stages
+constexpr int kSB = 2;        // xt chunk stages per slot
 constexpr int kABytes = 4096; // one tile row of A (128 channels x 16 k, fp16)
 constexpr int kABuf = 2;      // A stages per decoder (double buffered)
 constexpr int kMaxCtas = 148;
@@ -79,11 +80,12 @@ struct TcLayout {
     static constexpr int TMEM_COLS = kIssuers * 2 * NT;     // issuers x buffers x NT columns
     static constexpr int off_a = 0;                          // kABuf x kDecWarps A stages
     static constexpr int off_b = off_a + kABuf * kDecWarps * kABytes;
-    static constexpr int off_p = off_b + kSB * BBYTES;
+    static constexpr int off_p = off_b + kIssuers * kSB * BBYTES;
     static constexpr int off_z = off_p + kDecWarps * kRing * ROWB;
     static constexpr int off_bar = off_z + NT * 128 * 4;
-    // pfull[dec][ring], afull[slot][buf], aempty[slot][buf], bfull[SB], bempty[SB], dfull[iss][2], dempty[iss][2]
-    static constexpr int nbar = kDecWarps * kRing + 2 * kIssuers * kABuf + 2 * kSB + 4 * kIssuers;
+    // pfull[dec][ring], pempty[dec][ring], afull[slot][buf], aempty[slot][buf], bfull[slot][SB],
+    // bempty[slot][SB], dfull[iss][2], dempty[iss][2]
+    static constexpr int nbar = 2 * kDecWarps * kRing + 2 * kIssuers * kABuf + 2 * kIssuers * kSB + 4 * kIssuers;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
     static_assert(off_b % 1024 == 0 && off_p % 16 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
@@ -131,6 +133,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t sleep_ns = 0)
 {
+    // fast path: the phase is usually complete already -- one check per lane
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     int ok = 0;
     if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, abort_flag, sleep_ns) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -247,12 +251,13 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-    uint64_t* pfull = bar;                                   // [kDecWarps][kRing]
-    uint64_t* afull = pfull + kDecWarps * kRing;             // [slot][buf]: the 4 decoders of a slot arrive
+    uint64_t* pfull = bar;                                   // [kDecWarps][kRing]: packed words landed
+    uint64_t* pempty = pfull + kDecWarps * kRing;            // [kDecWarps][kRing]: decoder has read them
+    uint64_t* afull = pempty + kDecWarps * kRing;            // [slot][buf]: the 4 decoders of a slot arrive
     uint64_t* aempty = afull + kIssuers * kABuf;             // [slot][buf]: the slot's issuer commits
-    uint64_t* bfull = aempty + kIssuers * kABuf;             // [kSB]
-    uint64_t* bempty = bfull + kSB;                          // [kSB]
-    uint64_t* dfull = bempty + kSB;                          // [kIssuers][2]
+    uint64_t* bfull = aempty + kIssuers * kABuf;             // [slot][kSB]
+    uint64_t* bempty = bfull + kIssuers * kSB;               // [slot][kSB]
+    uint64_t* dfull = bempty + kIssuers * kSB;               // [kIssuers][2]
     uint64_t* dempty = dfull + 2 * kIssuers;                 // [kIssuers][2]
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort, [2] last-CTA flag
     volatile int* abort_flag = misc + 1;
@@ -269,9 +274,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     const int g_first = (int)(b0 / C), c_first = (int)(b0 % C);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kDecWarps * kRing; ++i) mbar_init(&pfull[i], 1);
+        for (int i = 0; i < kDecWarps * kRing; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], 1); }
         for (int i = 0; i < kIssuers * kABuf; ++i) { mbar_init(&afull[i], 4); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
+        for (int i = 0; i < kIssuers * kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
         for (int i = 0; i < 2 * kIssuers; ++i) { mbar_init(&dfull[i], 1); mbar_init(&dempty[i], kEpiWarps); }
         misc[1] = 0;
         misc[2] = 0;
@@ -286,16 +291,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
 
-    if (warp == 0) {
-        // ------------------------------------------- xt chunk producer ---
+    if (warp < kWarpIss0) {
+        // ------------------------------------------------------ producers ---
+        // Producer s issues, for each unit u = s (mod 4) of this CTA, the
+        // packed words of its 4 tile rows (one bulk copy into the ring of each
+        // decoder of slot s) and its xt chunk (into the slot's xt ring).
         if (lane == 0) {
-            int c = c_first;
-            for (int u = 0; u < n; ++u, ++c) {
-                if (c == C) c = 0;
-                const int bs = u % kSB;
-                if (!wait_or_abort(&bempty[bs], ((u / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
+            const int sl = warp - kWarpProd0;
+            int g = g_first, c = c_first + sl;
+            while (c >= C) { c -= C; ++g; }
+            for (int u = sl, k = 0; u < n; u += 4, ++k) {
+                const int rs = k % kRing;
+                const uint32_t rpar = ((k / kRing) & 1) ^ 1;
+                bool ok = true;
+#pragma unroll
+                for (int t = 0; t < 4 && ok; ++t) {
+                    const int d = sl * 4 + t;
+                    ok = wait_or_abort(&pempty[d * kRing + rs], rpar, abort_flag, kSleepNs);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&pfull[d * kRing + rs], L::ROWB);
+                    bulk_g2s(smem + L::off_p + (size_t)(d * kRing + rs) * L::ROWB,
+                             a.packed + ((size_t)(4 * c + t) * tiles_n + 8 * (size_t)g) * TW, L::ROWB,
+                             &pfull[d * kRing + rs]);
+                }
+                if (!ok) break;
+                const int bs = sl * kSB + k % kSB;
+                if (!wait_or_abort(&bempty[bs], ((k / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
                 mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
                 bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)c * L::BBYTES, L::BBYTES, &bfull[bs]);
+                c += 4;
+                while (c >= C) { c -= C; ++g; }
             }
         }
     } else if (warp < kWarpEpi0) {
@@ -319,7 +344,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                     const int k = u >> 2, ab = k & 1;            // k-th unit of slot i, A buffer
                     if (!wait_or_abort(&afull[i * kABuf + ab], (k >> 1) & 1, abort_flag, kIssSleepNs)) { ok = false; break; }
                     tc_fence_after();
-                    const int bs = u % kSB;
+                    const int bs = i * kSB + k % kSB;
                     const uint32_t bbase = smem_u32(smem + L::off_b + bs * L::BBYTES);
 #pragma unroll
                     for (int t = 0; t < 4; ++t) {
@@ -437,7 +462,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     } else {
         // ------------------------------------------------------ decoders ---
         const int d = warp - kWarpDec0;           // 0..15
-        const int slot = d >> 2, t = d & 3;       // units u = slot (mod 4); tile row t of each
+        const int slot = d >> 2;                  // units u = slot (mod 4); tile row d % 4 of each
         const int j = lane >> 2, q = lane & 3;
         const int src_prev = (lane & ~3) | ((q + 3) & 3);
         uint32_t soff[2][2];
@@ -449,30 +474,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
                 for (int e = 0; e < 2; ++e)
                     soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
         }
-        uint8_t* ring = smem + L::off_p + (size_t)d * kRing * L::ROWB;
-        uint64_t* myfull = pfull + d * kRing;
+        const uint8_t* ring = smem + L::off_p + (size_t)d * kRing * L::ROWB;
         const uint32_t ast0 = smem_u32(smem + L::off_a + d * kABytes);  // stage d (+ kDecWarps for buffer 1)
         const int nk = n > slot ? (n - slot + 3) / 4 : 0;      // units this decoder handles
-        // (block, chunk) of the next unit to prefetch, walked by steps of 4
-        // units (no division per unit)
-        int pf_g = g_first, pf_c = c_first + slot;
-        while (pf_c >= C) { pf_c -= C; ++pf_g; }
-        auto next_src = [&]() -> const uint32_t* {
-            const uint32_t* src = a.packed + ((size_t)(4 * pf_c + t) * tiles_n + 8 * (size_t)pf_g) * TW;
-            pf_c += 4;
-            while (pf_c >= C) { pf_c -= C; ++pf_g; }
-            return src;
-        };
-        if (lane == 0) {
-            for (int k = 0; k < kRing && k < nk; ++k) {
-                mbar_arrive_expect_tx(&myfull[k], L::ROWB);
-                bulk_g2s(ring + k * L::ROWB, next_src(), L::ROWB, &myfull[k]);
-            }
-        }
-        int k = 0;
-        for (; k < nk; ++k) {
+        for (int k = 0; k < nk; ++k) {
             const int rs = k % kRing;
-            if (!warp_wait(&myfull[rs], (k / kRing) & 1, abort_flag, kSleepNs)) break;
+            if (!warp_wait(&pfull[d * kRing + rs], (k / kRing) & 1, abort_flag, kSleepNs)) break;
             const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + rs * L::ROWB) + j * TW + q * QW;
             uint32_t buf[QW + 1];
             if constexpr (QW % 4 == 0) {
@@ -490,26 +497,16 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
             }
             buf[0] = __shfl_sync(0xffffffffu, buf[QW], src_prev);
             __syncwarp();
-            if (lane == 0 && k + kRing < nk) {
-                fence_proxy_async_smem();
-                mbar_arrive_expect_tx(&myfull[rs], L::ROWB);
-                bulk_g2s(ring + rs * L::ROWB, next_src(), L::ROWB, &myfull[rs]);
-            }
+            if (lane == 0) mbar_arrive(&pempty[d * kRing + rs]);      // slot free for the producer
             const int ab = k & 1;
             if (!warp_wait(&aempty[slot * kABuf + ab], ((k >> 1) & 1) ^ 1, abort_flag, kSleepNs)) break;
             decode_quarter_to_a<BITS>(buf, ast0 + ab * kDecWarps * kABytes, soff);
             fence_proxy_async_smem();
             // the unit's xt chunk must have landed before its MMAs are issued;
-            // the decoder checks it here so that the issuers wait only on afull
-            const int ub = 4 * k + slot;
-            if (!warp_wait(&bfull[ub % kSB], (ub / kSB) & 1, abort_flag, kSleepNs)) break;
+            // the decoder checks it here so that the issuer waits only on afull
+            if (!warp_wait(&bfull[slot * kSB + k % kSB], (k / kSB) & 1, abort_flag, kSleepNs)) break;
             __syncwarp();
             if (lane == 0) mbar_arrive(&afull[slot * kABuf + ab]);
-        }
-        // after an abort, let this warp's copies still in flight land before exit
-        if (k < nk && lane == 0) {
-            for (int kk = k; kk < nk && kk <= k + kRing; ++kk)
-                (void)mbar_wait_bounded(&myfull[kk % kRing], (kk / kRing) & 1, 100000000ull);
         }
     }
 
