@@ -72,7 +72,7 @@ int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* s
     a.n_out = n_out;
     a.bits = bits;
     a.ws = static_cast<unsigned char*>(ws);
-    cudaError_t e = m == 1 ? exl3::launch_gemv_cc(a, static_cast<cudaStream_t>(stream))
+    cudaError_t e = m == 1 ? exl3::launch_gemv_m1(a, static_cast<cudaStream_t>(stream))
                            : exl3::launch_gemm_tc(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }
@@ -103,13 +103,13 @@ int exl3_version(void) { return 100; }
 size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
     if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
-    return m == 1 ? exl3::cc_workspace_bytes(m, k_in, n_out, bits) : exl3::tc_workspace_bytes(m, k_in, n_out, bits);
+    return m == 1 ? exl3::m1_workspace_bytes(k_in, n_out, bits) : exl3::tc_workspace_bytes(m, k_in, n_out, bits);
 }
 
 int exl3_kernel_launches(int m, int k_in, int n_out, int bits)
 {
     if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
-    return m == 1 ? exl3::cc_launches(m) : 2;
+    return m == 1 ? 1 : 2;
 }
 
 int exl3_workspace_status(void* workspace, void* stream)
@@ -243,6 +243,6 @@ extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, cons
     a.n_out = n_out;
     a.bits = bits;
     a.ws = static_cast<unsigned char*>(ws);
-    e = exl3::launch_gemv_cc(a, s);
+    e = exl3::launch_gemv_m1(a, s);
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }

@@ -18,10 +18,18 @@ namespace exl3 {
 // 3INST: x = state*89226354 + 64248484 (mod 2^32), then
 // (x & 0x8FFF8FFF) ^ 0x3B603B60.  The result holds two fp16 values (low and
 // high halves) whose sum is the weight.
+// Written as one multiply-add and one three-input logic op (LUT 0x6A =
+// (a & b) ^ c); left to itself the compiler spends an extra integer
+// instruction on the two 32-bit constants.
 __device__ __forceinline__ uint32_t inst3(uint32_t state)
 {
-    const uint32_t x = state * 89226354u + 64248484u;
-    return (x & 0x8FFF8FFFu) ^ 0x3B603B60u;
+    uint32_t m;
+    asm("{\n\t.reg .b32 t;\n\t"
+        "mad.lo.u32 t, %1, 89226354, 64248484;\n\t"
+        "lop3.b32 %0, t, 0x8FFF8FFF, 0x3B603B60, 0x6A;\n\t}"
+        : "=r"(m)
+        : "r"(state));
+    return m;
 }
 
 // State whose 16-bit window starts P bits after the most significant bit of

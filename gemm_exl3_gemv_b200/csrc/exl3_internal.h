@@ -24,11 +24,9 @@ struct GemmArgs {
     unsigned char* ws;        // workspace base
 };
 
-// Split-K factor the CUDA-core kernel uses for this problem (host-only).
-int cc_splits(int m, int k_in, int n_out, int bits);
-size_t cc_workspace_bytes(int m, int k_in, int n_out, int bits);
-int cc_launches(int m);
-cudaError_t launch_gemv_cc(const GemmArgs& a, cudaStream_t stream);
+// Single-row product on CUDA cores (gemv_m1.cu).
+size_t m1_workspace_bytes(int k_in, int n_out, int bits);
+cudaError_t launch_gemv_m1(const GemmArgs& a, cudaStream_t stream);
 
 // Tensor-core path (2..32 rows): CTA count, workspace size, launcher (two
 // launches per call: input rotation pre-pass and the product kernel).
