@@ -60,12 +60,120 @@ __device__ __forceinline__ __half weight_of(uint32_t m)
 // high half): the low halves and the high halves of the two 3INST words are
 // gathered with byte permutes and added in one packed fp16 add (RNE), which
 // gives the same bits as weight_of on each word.
+// Same result, another instruction mix: each word's halves are added by one
+// half-precision add (operand halves selected in the instruction), and the
+// two sums are then packed -- more FMA-pipe and fewer integer-pipe work.
+__device__ __forceinline__ uint32_t weight_pair_h(uint32_t ma, uint32_t mb)
+{
+    uint32_t r;
+    asm("{\n\t.reg .f16 al, ah, bl, bh, wa, wb;\n\t"
+        "mov.b32 {al, ah}, %1;\n\t"
+        "mov.b32 {bl, bh}, %2;\n\t"
+        "add.rn.f16 wa, al, ah;\n\t"
+        "add.rn.f16 wb, bl, bh;\n\t"
+        "mov.b32 %0, {wa, wb};\n\t}"
+        : "=r"(r)
+        : "r"(ma), "r"(mb));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t weight_pair(uint32_t ma, uint32_t mb)
 {
     const uint32_t lo = __byte_perm(ma, mb, 0x5410);   // (ma[15:0], mb[15:0])
     const uint32_t hi = __byte_perm(ma, mb, 0x7632);   // (ma[31:16], mb[31:16])
     __half2 s = __hadd2(*reinterpret_cast<const __half2*>(&lo), *reinterpret_cast<const __half2*>(&hi));
     return *reinterpret_cast<uint32_t*>(&s);
+}
+
+// Isolate the 16-bit window that starts P bits after the most significant bit
+// of buf[0] (P a compile-time constant).  Windows at the top or bottom half
+// of a word take one instruction.  Otherwise ALT selects the form:
+//   ALT = false: shift right + mask (two integer-pipe instructions);
+//   ALT = true : shift left so the window is the top half, then a high
+//                multiply by 2^16 (`two16` is a runtime value, so the
+//                multiply stays on the FMA pipe) -- one integer-pipe and one
+//                FMA-pipe instruction.
+template <int P, int NW, bool ALT>
+__device__ __forceinline__ uint32_t window_of(const uint32_t (&buf)[NW], uint32_t two16)
+{
+    constexpr int wi = P >> 5, off = P & 31;
+    static_assert(wi + (off > 16 ? 1 : 0) < NW, "window outside the buffer");
+    if constexpr (off == 0) {
+        return buf[wi] >> 16;
+    } else if constexpr (off == 16) {
+        return buf[wi] & 0xFFFFu;
+    } else if constexpr (!ALT) {
+        if constexpr (off < 16) return (buf[wi] >> (16 - off)) & 0xFFFFu;
+        else return __funnelshift_r(buf[wi + 1], buf[wi], 48 - off) & 0xFFFFu;
+    } else {
+        uint32_t v;
+        if constexpr (off < 16) v = buf[wi] << off;
+        else v = __funnelshift_l(buf[wi + 1], buf[wi], off);
+        return __umulhi(v, two16);
+    }
+}
+
+// Byte-aligned variant for even bit widths: a window whose offset is r bits
+// (r = off mod 8) past a byte boundary is read from the stream shifted left
+// by r bits (one funnel shift per word, shared by every window of that word
+// with the same r), where it sits at a byte boundary: top half (shift), bytes
+// 1-2 (byte permute with zero fill) or bottom half (mask) -- one instruction.
+// Windows that straddle the next word fall back to window_of.
+template <int P, int NW>
+__device__ __forceinline__ uint32_t window_bytes(const uint32_t (&buf)[NW], uint32_t two16)
+{
+    constexpr int wi = P >> 5, off = P & 31, r = off & 7, ob = off - r;
+    if constexpr (ob == 24 || (r != 0 && wi + 1 >= NW)) {
+        return window_of<P, NW, false>(buf, two16);
+    } else {
+        uint32_t w;
+        if constexpr (r == 0) w = buf[wi];
+        else w = __funnelshift_l(buf[wi + 1], buf[wi], r);
+        if constexpr (ob == 0) return w >> 16;
+        else if constexpr (ob == 8) return __byte_perm(w, 0u, 0x4421);
+        else return w & 0xFFFFu;
+    }
+}
+
+
+// Window isolation chosen per bit width (measured on B200): byte-aligned
+// reads from shifted words for 2 and 4 bits; for 3 bits (windows at every
+// bit offset) every second non-aligned window on the FMA pipe.  R is the
+// weight's index in the run, P its window's start bit in `buf`.
+template <int BITS, int R, int P, int NW>
+__device__ __forceinline__ uint32_t window_auto(const uint32_t (&buf)[NW], uint32_t two16)
+{
+    if constexpr (BITS == 3) return window_of<P, NW, (R % 2) == 0>(buf, two16);
+    else return window_bytes<P, NW>(buf, two16);
+}
+
+// A lane's share of one tile row of a 128-channel block: 2*BITS consecutive
+// words at `src` (streaming loads: each word is read once).  K = 2, 4: 128-bit
+// loads; K = 3: 64-bit loads (the lane's 24 bytes are 8-byte aligned).
+template <int BITS>
+__device__ __forceinline__ void load_lane_words(uint32_t (&w)[2 * BITS], const uint32_t* src)
+{
+    if constexpr (BITS == 3) {
+#pragma unroll
+        for (int t = 0; t < 3; ++t) {
+            uint2 v;
+            asm volatile("ld.global.cs.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(src + 2 * t));
+            w[2 * t] = v.x;
+            w[2 * t + 1] = v.y;
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < BITS / 2; ++t) {
+            uint4 v;
+            asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "l"(src + 4 * t));
+            w[4 * t] = v.x;
+            w[4 * t + 1] = v.y;
+            w[4 * t + 2] = v.z;
+            w[4 * t + 3] = v.w;
+        }
+    }
 }
 
 }  // namespace exl3

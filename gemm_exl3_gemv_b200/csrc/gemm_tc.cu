@@ -1,45 +1,41 @@
 // gemm_tc.cu -- the verify-batch product (2..32 input rows) on the 5th-generation
 // tensor cores (tcgen05), with the trellis decode on the CUDA cores.
 //
-// What is computed (the "WMMA GEMV for draft verification" / "batched
-// verification up to 32 rows" the exl3-rdna4-recipe page describes in "What we
+// What is computed (the "WMMA GEMV for draft verification" and "batched
+// verification up to 32 rows" of the exl3-rdna4-recipe page, section "What we
 // added on top of upstream", here on B200):
 //     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: m x K_in, y: m x N_out
 //
-// Design (each choice measured on B200):
-//   * A pre-pass writes xt = H(su .* x) once per call, fp16, already laid out
-//     as the MMA's B operand (K-major, 128-byte swizzle), m padded to NT = 16
-//     or 32 rows with zeros.
-//   * Work unit = one 64-row chunk of K_in for one 128-channel output block
-//     (4 tile rows, 8192 weights).  Persistent stream-K grid: the G x C units
-//     are cut into equal contiguous ranges, at most one CTA per SM.  A range
-//     may cover the end of one block and the start of the next; each
-//     (CTA, block) piece is a segment.
-//   * Decode straight into the A operand: the two fp16 halves of each 3INST
-//     word are kept as two adjacent A rows (lo, hi) of the same input row k,
-//     so the decoded 32-bit word is stored as is and the tensor core adds the
-//     halves.  A is M = 128 rows (64 channels x lo/hi) by K = 16, MN-major with
-//     the 128-byte swizzle; one tile row gives two MMAs (channels 0-63,
-//     64-127).  The 16 k of a tile row are permuted (the same permutation is
-//     applied to xt) so that the 16-byte stores of a warp hit distinct banks.
-//   * 16 decoder warps (4 per scheduler, enough to keep the integer pipes
-//     busy); decoder d always decodes tile row d%4 of the units u = d/4
-//     (mod 4) into its own A stage and fetches its own packed words with 1-D bulk copies into a
-//     private 3-slot ring -- bulk-copy issue costs ~85 ns per copy per thread,
-//     so it is spread over 16 threads.
-//   * 4 MMA-issuing threads (one per warp).  A thread that waits on a barrier
-//     right after issuing MMAs stalls until they drain (~0.1 us), so a single
-//     issuer cannot keep the tensor core busy; issuer i takes every unit
-//     u = i (mod 4) (8 MMAs per barrier wait) into its own accumulator, the
-//     four interleave on the tensor core, and the epilogue adds the four
-//     accumulators in a fixed order.
-//   * Accumulators in tensor memory: 4 issuers x 2 buffers x 2 channel halves
-//     x NT fp32 columns; a segment is drained while the next accumulates.
-//     Segments of a block are combined by the last CTA to finish (arrival
-//     counter) in segment order -- fixed, so results are bitwise repeatable --
-//     which then scales, rotates and writes y.
-//   * Every wait is bounded (2 s); on expiry the CTA records a timeout in the
-//     workspace status word and winds down.
+// Design:
+//   * A pre-pass writes xt = H(su .* x) once per call into the workspace, fp16,
+//     laid out as the MMA's B operand (K-major, 128-byte swizzle), m padded to
+//     NT = 16 or 32 rows with zeros.
+//   * Unit = one 128-row block of K_in for one 128-channel output block: 8
+//     tile rows, 16384 weights.  Stream-K: the G x C units are cut into equal
+//     contiguous ranges, one per CTA, two CTAs per SM.  A range may cover the
+//     end of one block and the start of the next; each (CTA, block) piece is
+//     a segment.
+//   * Eight decoder warps.  Warp w decodes tile row w of every unit: lane l
+//     takes quarter l%4 of tile l/4 (64 consecutive weights) from its words,
+//     loaded straight from HBM into registers one unit ahead (coalesced: the
+//     warp reads the tile row's 256*K contiguous bytes).  The two fp16 halves
+//     of each 3INST word are added once (RNE: the exact decoded weight) and
+//     stored into the warp's own A stage (128 channels x 16 k, MN-major,
+//     128-byte swizzle).  Lane 0 of the warp then issues the MMA itself --
+//     tcgen05.mma kind::f16, M = 128 channels, N = NT rows, K = 16 -- into the
+//     warp's own tensor-memory accumulator, and commits it to the stage's
+//     barrier.  No dedicated issuer warps and no polling: a warp waits only
+//     for its own stage (two units back) and for the unit's xt chunk.
+//   * A ninth warp streams the xt chunks (1-D bulk copies + mbarrier) into a
+//     two-stage ring shared by the eight decoders.
+//   * End of a segment: every warp reads its lane quarter of all eight
+//     accumulators (tcgen05.ld) and adds them in a fixed order.  A block
+//     split over several CTAs: each writes its partial sums to the workspace
+//     and the last to arrive (atomic counter, no waiting) adds them in CTA
+//     order -- fixed, so results are bitwise repeatable -- then scales,
+//     rotates and writes y.
+//   * Every mbarrier wait is bounded (2 s); on expiry the CTA records a
+//     timeout in the workspace status word and winds down.
 #include <atomic>
 #include <utility>
 
@@ -52,45 +48,35 @@ namespace exl3 {
 
 namespace {
 
-constexpr int kDecWarps = 16;
-constexpr int kIssuers = 4;
-constexpr int kEpiWarps = 4;
-constexpr int kWarpProd0 = 0;                         // warps 0..3 issue the bulk copies of slots 0..3
-constexpr int kWarpIss0 = 4;                          // warps 4..7 issue MMAs
-constexpr int kWarpEpi0 = kWarpIss0 + kIssuers;       // warps 8..11 drain accumulators
-constexpr int kWarpDec0 = kWarpEpi0 + kEpiWarps;      // warps 12..27 decode
-constexpr int kTcWarps = kWarpDec0 + kDecWarps;
-constexpr int kTcThreads = 32 * kTcWarps;
-constexpr int kRing = 3;      // packed-word slots per decoder
-constexpr int kSB = 2;        // xt chunk stages per slot
-constexpr int kABytes = 4096; // one tile row of A (128 channels x 16 k, fp16)
-constexpr int kABuf = 2;      // A stages per decoder (double buffered)
-constexpr int kMaxCtas = 148;
-constexpr int kMinUnitsPerCta = 10;
-// Suspend hints for barrier waits (ns): waiting threads are parked in
-// hardware instead of polling, leaving the issue slots to the decoders.
-constexpr uint32_t kSleepNs = 2000;
-constexpr uint32_t kIssSleepNs = 1000;
-constexpr uint32_t kEpiSleepNs = 20000;
+constexpr int kDec = 8;                        // decoder warps (one accumulator each)
+constexpr int kProdWarp = kDec;                // warp 8: xt chunk producer
+constexpr int kTcThreads = 32 * (kDec + 1);
+constexpr int kAStages = 2;                    // A stages per decoder warp
+constexpr int kBStages = 4;                    // xt unit stages (shared by the eight decoders)
+constexpr int kABytes = 4096;                  // one tile row of A: 128 channels x 16 k, fp16
+constexpr int kCtasPerSm = 2;
+constexpr int kSms = 148;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <int BITS, int NT>
+template <int NT>
 struct TcLayout {
-    static constexpr int ROWB = 256 * BITS;                 // packed bytes per tile row
-    static constexpr int BBYTES = NT * 128;                 // xt bytes per 64-row chunk
-    static constexpr int TMEM_COLS = kIssuers * 2 * NT;     // issuers x buffers x NT columns
-    static constexpr int off_a = 0;                          // kABuf x kDecWarps A stages
-    static constexpr int off_b = off_a + kABuf * kDecWarps * kABytes;
-    static constexpr int off_p = off_b + kIssuers * kSB * BBYTES;
-    static constexpr int off_z = off_p + kDecWarps * kRing * ROWB;
-    static constexpr int off_bar = off_z + NT * 128 * 4;
-    // pfull[dec][ring], pempty[dec][ring], afull[slot][buf], aempty[slot][buf], bfull[slot][SB],
-    // bempty[slot][SB], dfull[iss][2], dempty[iss][2]
-    static constexpr int nbar = 2 * kDecWarps * kRing + 2 * kIssuers * kABuf + 2 * kIssuers * kSB + 4 * kIssuers;
+    static constexpr int CHUNK = NT * 128;                    // xt bytes per 64 input rows
+    static constexpr int BUNIT = 2 * CHUNK;                   // xt bytes per unit (128 rows)
+    static constexpr int TMEM_COLS = kDec * NT;               // one NT-column accumulator per decoder
+    static constexpr int off_a = 0;                           // [kDec][kAStages] A stages
+    static constexpr int off_z = off_a;                       // z [NT][128] fp32, over the A stages (segment end)
+    static constexpr int off_b = off_a + kDec * kAStages * kABytes;
+    static constexpr int off_bar = off_b + kBStages * BUNIT;
+    // aempty[kDec][kAStages], bfull[kBStages], bempty[kBStages], segdone
+    static constexpr int nbar = kDec * kAStages + 2 * kBStages + 1;
     static constexpr int off_misc = off_bar + nbar * 8;
-    static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
-    static_assert(off_b % 1024 == 0 && off_p % 16 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
-    static_assert(TMEM_COLS >= 32 && TMEM_COLS <= 512, "tensor memory");
-    static_assert(total <= 227 * 1024, "shared memory");
+    static constexpr int total = off_misc + 64 + 1024;       // + slack to align the base to 1024
+    static_assert(off_b % 1024 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
+    static_assert(NT * 128 * 4 <= kDec * kAStages * kABytes, "z fits over the A stages");
+    static_assert(TMEM_COLS == 128 || TMEM_COLS == 256, "tensor memory (power of two, two CTAs per SM)");
+    // at most two CTAs fit on an SM, so their accumulators always fit in its 512 columns
+    static_assert(3 * total > 227 * 1024, "a third CTA per SM must not fit");
+    static_assert(kCtasPerSm * total <= 227 * 1024, "two CTAs per SM");
 };
 
 struct TcParams {
@@ -99,8 +85,9 @@ struct TcParams {
     float* part;            // segment partial sums, [slot][NT][128]
     uint32_t* counters;     // per output block
     uint32_t* status;       // workspace status word
-    int G, C, P;            // output blocks, 64-row chunks per block, CTAs
+    int G, C, P;            // output blocks, 128-row input blocks, CTAs
     long long U;            // units = G * C
+    uint32_t two16;         // 2^16, passed at run time (keeps a multiply on the FMA pipe)
 };
 
 __host__ __device__ inline int cta_of_unit(long long x, int P, long long U)
@@ -108,79 +95,43 @@ __host__ __device__ inline int cta_of_unit(long long x, int P, long long U)
     return (int)(((x + 1) * P - 1) / U);
 }
 
-// Bounded wait; also gives up early once another role has aborted.  With
-// sleep_ns > 0 the thread may be suspended in hardware between checks (it is
-// resumed when the phase completes).
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              uint32_t sleep_ns = 0)
+// Bounded wait on one thread; gives up early once another thread has aborted.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     while (true) {
-        for (int i = 0; i < 8; ++i) {
-            if (sleep_ns ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity)) return true;
-        }
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait_sleep(bar, parity, 1000)) return true;
         if (*abort_flag) return false;
-        if (global_ns() - t0 > 2000000000ull) {
+        if (global_ns() - t0 > kWaitLimitNs) {
             atomicExch((int*)abort_flag, 1);
             return false;
         }
     }
 }
 
-// Warp-wide wait: lane 0 polls, the outcome is broadcast, then every lane
-// observes the completed phase once itself (acquire for each thread).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t sleep_ns = 0)
+// Warp-wide wait: every lane observes the completed phase (acquire per lane).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
 {
-    // fast path: the phase is usually complete already -- one check per lane
     if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
     int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, abort_flag, sleep_ns) ? 1 : 0;
+    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, abort_flag) ? 1 : 0;
     ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (ok) {
-        // the phase has completed and cannot advance again before this warp
-        // acts on it, so this succeeds at once; bounded all the same
-        int tries = 0;
-        while (!mbar_try_wait(bar, parity) && ++tries < (1 << 20)) {
-        }
-        ok = __all_sync(0xffffffffu, tries < (1 << 20)) ? 1 : 0;
-        if (!ok && (threadIdx.x & 31) == 0) atomicExch((int*)abort_flag, 1);
+    if (!ok) return false;
+    // the phase has completed and cannot advance again before this warp acts
+    // on it, so this succeeds at once; bounded all the same
+    int tries = 0;
+    while (!mbar_try_wait(bar, parity) && ++tries < (1 << 20)) {
     }
+    ok = __all_sync(0xffffffffu, tries < (1 << 20)) ? 1 : 0;
+    if (!ok && (threadIdx.x & 31) == 0) atomicExch((int*)abort_flag, 1);
     return ok != 0;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
 {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-// Decode the 64 weights of quarter q of tile j (4 input rows x 16 channels)
-// into fp16 (the two halves of each 3INST word added and rounded once, RNE:
-// the exact decoded weight) and store them into the A stage at `ast`, two
-// 16-byte chunks per row.  soff[rb][e]: per-lane byte offset of the chunk
-// holding channels 8e..8e+7 of a row with (row & 1) == rb; row >> 1 selects
-// the 8-row K group (+2048 bytes).
-template <int BITS, int NW>
-__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast, const uint32_t (&soff)[2][2])
-{
-    // fully unrolled over (row r, chunk e): every window position is a compile-time constant
-    auto body = [&](auto R, auto E) {
-        constexpr int r = decltype(R)::value, e = decltype(E)::value;
-        // channels 8e + 2c, 8e + 2c + 1 of row r -> one fp16 pair
-        auto pair = [&](auto Cc) -> uint32_t {
-            constexpr int c = decltype(Cc)::value;
-            const uint32_t ma = inst3(window16<(16 * r + 8 * e + 2 * c + 1) * BITS + 16>(buf));
-            const uint32_t mb = inst3(window16<(16 * r + 8 * e + 2 * c + 2) * BITS + 16>(buf));
-            return weight_pair(ma, mb);
-        };
-        sts128(ast + soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
-               pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
-               pair(std::integral_constant<int, 3>{}));
-    };
-    [&]<int... RE>(std::integer_sequence<int, RE...>) {
-        (body(std::integral_constant<int, RE / 2>{}, std::integral_constant<int, RE % 2>{}), ...);
-    }(std::make_integer_sequence<int, 8>{});
 }
 
 // Row v of an accumulator (row v of A) holds output channel chan_of_row(v):
@@ -195,70 +146,95 @@ __device__ __forceinline__ int chan_of_row(int v)
     return 16 * (4 * atom + j4) + 8 * (chunk & 1) + pos;
 }
 
+// Decode the 64 weights of quarter q of tile j (4 input rows x 16 channels)
+// into fp16 (the two halves of each 3INST word added and rounded once, RNE:
+// the exact decoded weight) and store them into the A stage at `ast`, two
+// 16-byte chunks per row.  soff[rb][e]: per-lane byte offset of the chunk
+// holding channels 8e..8e+7 of a row with (row & 1) == rb; row >> 1 selects
+// the 8-row K group (+2048 bytes).
+template <int BITS, int NW>
+__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast,
+                                                    const uint32_t (&soff)[2][2], uint32_t two16)
+{
+    auto body = [&](auto R, auto E) {
+        constexpr int r = decltype(R)::value, e = decltype(E)::value;
+        // channels 8e + 2c, 8e + 2c + 1 of row r -> one fp16 pair
+        auto pair = [&](auto Cc) -> uint32_t {
+            constexpr int c = decltype(Cc)::value;
+            constexpr int ia = 16 * r + 8 * e + 2 * c, ib = ia + 1;
+            const uint32_t ma = inst3(window_auto<BITS, ia, (ia + 1) * BITS + 16>(buf, two16));
+            const uint32_t mb = inst3(window_auto<BITS, ib, (ib + 1) * BITS + 16>(buf, two16));
+            return weight_pair_h(ma, mb);
+        };
+        sts128(ast + soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
+               pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
+               pair(std::integral_constant<int, 3>{}));
+    };
+    [&]<int... RE>(std::integer_sequence<int, RE...>) {
+        (body(std::integral_constant<int, RE / 2>{}, std::integral_constant<int, RE % 2>{}), ...);
+    }(std::make_integer_sequence<int, 8>{});
+}
+
 // zsm[0 .. m*128) = sum of the partial slots (q + g) for q = p_first..p_last,
-// added in that order.  128 threads; each owns up to NT/4 float4 outputs and
-// keeps 2 x NT/4 independent loads in flight (a dependent chain of L2 loads
-// would take ~0.4 us per partial).
+// added in that order, by the 256 decoder threads.
 template <int NT>
 __device__ __forceinline__ void reduce_segments(const float* part, int g, int p_first, int p_last, int m, int et,
                                                 float* zsm)
 {
-    constexpr int F = NT / 4;                  // float4 outputs per thread, at most
-    float4 acc[F];
+    // thread et owns float4 outputs et + 256 i (i < NI); per step it loads one
+    // float4 of each of its outputs from two partials: 2 * NI loads in flight
+    constexpr int NI = NT / 8;                 // NT * 32 float4 outputs / 256 threads
     const int nf = m * 32;                     // float4 outputs in use
+    float4 acc[NI];
 #pragma unroll
-    for (int r = 0; r < F; ++r) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int i = 0; i < NI; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     int qq = p_first;
     for (; qq + 1 <= p_last; qq += 2) {
         const float4* s0 = reinterpret_cast<const float4*>(part + (size_t)(qq + g) * NT * 128);
         const float4* s1 = reinterpret_cast<const float4*>(part + (size_t)(qq + 1 + g) * NT * 128);
-        float4 v0[F], v1[F];
+        float4 v0[NI], v1[NI];
 #pragma unroll
-        for (int r = 0; r < F; ++r) {
-            const int f = et + 128 * r;
-            v0[r] = f < nf ? __ldcg(s0 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-            v1[r] = f < nf ? __ldcg(s1 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < NI; ++i) {
+            const int f = et + 32 * kDec * i;
+            v0[i] = f < nf ? __ldcg(s0 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            v1[i] = f < nf ? __ldcg(s1 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int r = 0; r < F; ++r) {
-            acc[r].x += v0[r].x; acc[r].y += v0[r].y; acc[r].z += v0[r].z; acc[r].w += v0[r].w;
-            acc[r].x += v1[r].x; acc[r].y += v1[r].y; acc[r].z += v1[r].z; acc[r].w += v1[r].w;
+        for (int i = 0; i < NI; ++i) {
+            acc[i].x += v0[i].x; acc[i].y += v0[i].y; acc[i].z += v0[i].z; acc[i].w += v0[i].w;
+            acc[i].x += v1[i].x; acc[i].y += v1[i].y; acc[i].z += v1[i].z; acc[i].w += v1[i].w;
         }
     }
     if (qq <= p_last) {
         const float4* s0 = reinterpret_cast<const float4*>(part + (size_t)(qq + g) * NT * 128);
 #pragma unroll
-        for (int r = 0; r < F; ++r) {
-            const int f = et + 128 * r;
+        for (int i = 0; i < NI; ++i) {
+            const int f = et + 32 * kDec * i;
             if (f < nf) {
                 const float4 v = __ldcg(s0 + f);
-                acc[r].x += v.x; acc[r].y += v.y; acc[r].z += v.z; acc[r].w += v.w;
+                acc[i].x += v.x; acc[i].y += v.y; acc[i].z += v.z; acc[i].w += v.w;
             }
         }
     }
 #pragma unroll
-    for (int r = 0; r < F; ++r) {
-        const int f = et + 128 * r;
-        if (f < nf) reinterpret_cast<float4*>(zsm)[f] = acc[r];
+    for (int i = 0; i < NI; ++i) {
+        const int f = et + 32 * kDec * i;
+        if (f < nf) reinterpret_cast<float4*>(zsm)[f] = acc[i];
     }
 }
 
 template <int BITS, int NT>
-__global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
+__global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParams prm)
 {
-    using L = TcLayout<BITS, NT>;
+    using L = TcLayout<NT>;
     constexpr int TW = 8 * BITS, QW = 2 * BITS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-    uint64_t* pfull = bar;                                   // [kDecWarps][kRing]: packed words landed
-    uint64_t* pempty = pfull + kDecWarps * kRing;            // [kDecWarps][kRing]: decoder has read them
-    uint64_t* afull = pempty + kDecWarps * kRing;            // [slot][buf]: the 4 decoders of a slot arrive
-    uint64_t* aempty = afull + kIssuers * kABuf;             // [slot][buf]: the slot's issuer commits
-    uint64_t* bfull = aempty + kIssuers * kABuf;             // [slot][kSB]
-    uint64_t* bempty = bfull + kIssuers * kSB;               // [slot][kSB]
-    uint64_t* dfull = bempty + kIssuers * kSB;               // [kIssuers][2]
-    uint64_t* dempty = dfull + 2 * kIssuers;                 // [kIssuers][2]
+    uint64_t* aempty = bar;                                   // [kDec][kAStages]: the stage's MMA completed
+    uint64_t* bfull = aempty + kDec * kAStages;               // [kBStages]: xt unit landed
+    uint64_t* bempty = bfull + kBStages;                      // [kBStages]: all 8 MMAs on it completed
+    uint64_t* segdone = bempty + kBStages;                    // every accumulator of the segment final
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort, [2] last-CTA flag
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
@@ -268,21 +244,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     const int p = blockIdx.x;
     const long long b0 = (long long)p * prm.U / prm.P;
     const long long b1 = (long long)(p + 1) * prm.U / prm.P;
-    const int n = (int)(b1 - b0);                            // units of this CTA
     const int C = prm.C;
     const int tiles_n = a.n_out / 16;
-    const int g_first = (int)(b0 / C), c_first = (int)(b0 % C);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kDecWarps * kRing; ++i) { mbar_init(&pfull[i], 1); mbar_init(&pempty[i], 1); }
-        for (int i = 0; i < kIssuers * kABuf; ++i) { mbar_init(&afull[i], 4); mbar_init(&aempty[i], 1); }
-        for (int i = 0; i < kIssuers * kSB; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], 1); }
-        for (int i = 0; i < 2 * kIssuers; ++i) { mbar_init(&dfull[i], 1); mbar_init(&dempty[i], kEpiWarps); }
+        for (int i = 0; i < kDec * kAStages; ++i) mbar_init(&aempty[i], 1);
+        for (int i = 0; i < kBStages; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kDec); }
+        mbar_init(segdone, kDec);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
     }
-    if (warp == kWarpIss0) {
+    if (warp == 0) {
         tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), L::TMEM_COLS);
         tmem_relinquish();
     }
@@ -291,229 +264,192 @@ __global__ void __launch_bounds__(kTcThreads, 1) gemm_tc_kernel(TcParams prm)
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
 
-    if (warp < kWarpIss0) {
-        // ------------------------------------------------------ producers ---
-        // Producer s issues, for each unit u = s (mod 4) of this CTA, the
-        // packed words of its 4 tile rows (one bulk copy into the ring of each
-        // decoder of slot s) and its xt chunk (into the slot's xt ring).
+    if (warp == kProdWarp) {
+        // ------------------------------------------------- xt producer ---
+        // xt of unit (g, c) is chunks 2c, 2c+1: BUNIT contiguous bytes.
         if (lane == 0) {
-            const int sl = warp - kWarpProd0;
-            int g = g_first, c = c_first + sl;
-            while (c >= C) { c -= C; ++g; }
-            for (int u = sl, k = 0; u < n; u += 4, ++k) {
-                const int rs = k % kRing;
-                const uint32_t rpar = ((k / kRing) & 1) ^ 1;
-                bool ok = true;
-#pragma unroll
-                for (int t = 0; t < 4 && ok; ++t) {
-                    const int d = sl * 4 + t;
-                    ok = wait_or_abort(&pempty[d * kRing + rs], rpar, abort_flag, kSleepNs);
-                    if (!ok) break;
-                    mbar_arrive_expect_tx(&pfull[d * kRing + rs], L::ROWB);
-                    bulk_g2s(smem + L::off_p + (size_t)(d * kRing + rs) * L::ROWB,
-                             a.packed + ((size_t)(4 * c + t) * tiles_n + 8 * (size_t)g) * TW, L::ROWB,
-                             &pfull[d * kRing + rs]);
-                }
-                if (!ok) break;
-                const int bs = sl * kSB + k % kSB;
-                if (!wait_or_abort(&bempty[bs], ((k / kSB) & 1) ^ 1, abort_flag, kSleepNs)) break;
-                mbar_arrive_expect_tx(&bfull[bs], L::BBYTES);
-                bulk_g2s(smem + L::off_b + bs * L::BBYTES, prm.xt + (size_t)c * L::BBYTES, L::BBYTES, &bfull[bs]);
-                c += 4;
-                while (c >= C) { c -= C; ++g; }
+            int kk = 0;
+            int c = (int)(b0 % C);
+            for (long long u = b0; u < b1; ++u, ++kk) {
+                const int s = kk & (kBStages - 1);
+                if (kk >= kBStages && !wait_or_abort(&bempty[s], (uint32_t)(kk / kBStages - 1) & 1u, abort_flag)) break;
+                mbar_arrive_expect_tx(&bfull[s], L::BUNIT);
+                bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
+                if (++c == C) c = 0;
+            }
+            // let every issued copy land before the CTA can exit
+            const int issued = kk;
+            for (int v = issued > kBStages ? issued - kBStages : 0; v < issued; ++v) {
+                if (*abort_flag)
+                    (void)mbar_wait_bounded(&bfull[v & (kBStages - 1)], (uint32_t)(v / kBStages) & 1u, 100000000ull);
             }
         }
-    } else if (warp < kWarpEpi0) {
-        // --------------------------------------------------- MMA issuers ---
-        // Issuer i takes the units u = i (mod 4) -- all 4 tile rows, 8 MMAs per
-        // barrier wait -- into its own accumulator.  It takes part in every
-        // segment (waits for its buffer, commits it) even when it has no unit
-        // there, so that every barrier sees one phase per segment.
-        if (lane == 0) {
-            const int i = warp - kWarpIss0;
-            constexpr uint32_t idesc = idesc_f16_amn(128, NT);
-            int seg = 0, u0 = 0, c0 = c_first;
-            bool ok = true;
-            while (ok && u0 < n) {
-                const int len = (n - u0) < (C - c0) ? (n - u0) : (C - c0);
-                const int db = seg & 1;
-                if (!wait_or_abort(&dempty[2 * i + db], ((seg >> 1) & 1) ^ 1, abort_flag, kIssSleepNs)) break;
-                const uint32_t dcol = tmem + (uint32_t)((i * 2 + db) * NT);
-                bool first = true;
-                for (int u = u0 + ((i - u0) & 3); u < u0 + len; u += 4) {
-                    const int k = u >> 2, ab = k & 1;            // k-th unit of slot i, A buffer
-                    if (!wait_or_abort(&afull[i * kABuf + ab], (k >> 1) & 1, abort_flag, kIssSleepNs)) { ok = false; break; }
-                    tc_fence_after();
-                    const int bs = i * kSB + k % kSB;
-                    const uint32_t bbase = smem_u32(smem + L::off_b + bs * L::BBYTES);
+
+    } else {
+    // ---- decoder warps: the segment loop (the producer never joins their
+    // barriers, which are the 256-thread named barrier 1) ----
+    const int j = lane >> 2, q = lane & 3;
+    const int src_prev = (lane & ~3) | ((q + 3) & 3);
+    uint32_t soff[2][2];
+    {
+        const int atom = j >> 2, j4 = j & 3;
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const uint32_t abase = smem_u32(smem + L::off_a + (ab * kDecWarps + i * 4 + t) * kABytes);
-                        mma_f16_ss(dcol, sdesc_sw128(abase, 1024, 2048), sdesc_sw128(bbase + t * 32, 16, 1024), idesc,
-                                   (first && t == 0) ? 0u : 1u);
-                    }
-                    first = false;
-                    mma_commit(&aempty[i * kABuf + ab]);
+        for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+            for (int e = 0; e < 2; ++e)
+                soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
+    }
+    constexpr uint32_t idesc = idesc_f16_amn(128, NT);
+    static_assert(kAStages == 2, "A stage index = unit counter & 1");
+    static_assert((kBStages & (kBStages - 1)) == 0, "power of two");
+    const uint32_t ast0 = smem_u32(smem + L::off_a + (warp * kAStages + 0) * kABytes);
+    const uint32_t ast1 = smem_u32(smem + L::off_a + (warp * kAStages + 1) * kABytes);
+    const uint64_t adesc0 = sdesc_sw128(ast0, 1024, 2048), adesc1 = sdesc_sw128(ast1, 1024, 2048);
+    // this warp's tile row is rows 16*warp .. +15 of the unit: chunk warp/4, 32 bytes per 16 rows
+    const uint32_t bw = (uint32_t)((warp >> 2) * L::CHUNK + (warp & 3) * 32);
+    // stage bs adds bs * BUNIT to the start address (no carry out of the 14-bit field: smem < 256 KB)
+    const uint64_t bdesc0 = sdesc_sw128(smem_u32(smem + L::off_b) + bw, 16, 1024);
+    const uint32_t dcol = tmem + (uint32_t)(warp * NT);
+    int kk = 0;                // unit counter of this CTA (stage and parity index)
+    int seg = 0;
+    for (long long u0 = b0; u0 < b1; ++seg) {
+        const int g = (int)(u0 / C);
+        const int c0 = (int)(u0 - (long long)g * C);
+        const long long u1 = ((long long)(g + 1) * C < b1) ? (long long)(g + 1) * C : b1;
+        const int nseg = (int)(u1 - u0);
+
+        {
+            // --------------------------------------------- decoder warp ---
+            const uint32_t* src = a.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
+            const size_t unit_step = (size_t)8 * tiles_n * TW;        // words between consecutive units
+            bool ok = true;
+            // decode unit k (the CTA's kk-th) from `wds` into A stage kk & 1, then
+            // lane 0 issues its MMA into this warp's accumulator
+            auto unit = [&](const uint32_t (&wds)[QW], int k, int kk) {
+                const int s = kk & (kAStages - 1), bs = kk & (kBStages - 1);
+                const uint32_t ph = (uint32_t)(kk / kAStages) & 1u, bph = (uint32_t)(kk / kBStages) & 1u;
+                if (kk >= kAStages && !warp_wait(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag)) ok = false;
+                if (!ok) return;
+                uint32_t buf[QW + 1];
+                buf[0] = __shfl_sync(0xffffffffu, wds[QW - 1], src_prev);
+#pragma unroll
+                for (int t = 0; t < QW; ++t) buf[t + 1] = wds[t];
+                decode_quarter_to_a<BITS>(buf, s ? ast1 : ast0, soff, prm.two16);
+                fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
+                __syncwarp();
+                if (lane == 0 && wait_or_abort(&bfull[bs], bph, abort_flag)) {
+                    tc_fence_after();
+                    const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);   // start address field
+                    mma_f16_ss(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
+                    mma_commit(&aempty[warp * kAStages + s]);
                     mma_commit(&bempty[bs]);
                 }
-                mma_commit(&dfull[2 * i + db]);
-                ++seg;
-                u0 += len;
-                c0 = 0;
+                ok = __shfl_sync(0xffffffffu, *abort_flag == 0 ? 1 : 0, 0) != 0;
+            };
+            uint32_t wa[QW], wb[QW];
+            load_lane_words<BITS>(wa, src);
+            int k = 0;
+            for (; k + 2 <= nseg; k += 2) {
+                load_lane_words<BITS>(wb, src + (size_t)(k + 1) * unit_step);
+                unit(wa, k, kk + k);
+                if (k + 2 < nseg) load_lane_words<BITS>(wa, src + (size_t)(k + 2) * unit_step);
+                unit(wb, k + 1, kk + k + 1);
+            }
+            if (k < nseg) unit(wa, k, kk + k);
+            kk += nseg;
+            if (lane == 0) {
+                if (ok) mma_commit(segdone);             // arrives once this warp's MMAs are done
+                else mbar_arrive(segdone);
             }
         }
-    } else if (warp < kWarpDec0) {
-        // ----------------------------------------------------- epilogue ---
-        const int ew = warp - kWarpEpi0;    // 0..3
-        const int quad = warp & 3;          // tensor-memory lanes 32*quad .. 32*quad+31
-        const int et = threadIdx.x - 32 * kWarpEpi0;   // 0..127
-        int seg = 0;
-        int u0 = 0, g = g_first, c0 = c_first;
-        while (u0 < n) {
-            const int len = (n - u0) < (C - c0) ? (n - u0) : (C - c0);
-            const int db = seg & 1;
-            bool ok = true;
-            for (int i = 0; i < kIssuers && ok; ++i)
-                ok = warp_wait(&dfull[2 * i + db], (seg >> 1) & 1, abort_flag, kEpiSleepNs);
-            if (!ok) break;
-            tc_fence_after();
-            {
-                const int v = 32 * quad + lane;
-                float acc[NT];
+
+        // ---- segment epilogue: accumulators -> zsm[NT][128] ----
+        bool ok = warp_wait(segdone, (uint32_t)(seg & 1), abort_flag);
+        tc_fence_after();
+        constexpr int kReaders = NT == 32 ? 8 : 4;         // warps reading the accumulators
+        if (warp < kReaders && ok) {
+            const int quad = warp & 3;                       // tensor-memory lanes 32*quad .. +31
+            const int tok0 = (warp >> 2) * 16;               // 16 rows (accumulator columns) per warp
+            float acc[16];
 #pragma unroll
-                for (int mm = 0; mm < NT; ++mm) acc[mm] = 0.f;
+            for (int t = 0; t < 16; ++t) acc[t] = 0.f;
 #pragma unroll
-                for (int i = 0; i < kIssuers; ++i) {
-                    if (len < 4 && ((i - u0) & 3) >= len) continue;   // issuer i had no unit here
+            for (int w = 0; w < kDec; ++w) {
+                uint32_t t16[16];
+                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(w * NT + tok0), t16);
+                tmem_ld_wait();
 #pragma unroll
-                    for (int cc = 0; cc < NT / 16; ++cc) {
-                        uint32_t t16[16];
-                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)((i * 2 + db) * NT + 16 * cc), t16);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) acc[16 * cc + e] += __uint_as_float(t16[e]);
-                    }
-                }
-                const int ch = chan_of_row(v);
-#pragma unroll
-                for (int mm = 0; mm < NT; ++mm) zsm[mm * 128 + ch] = acc[mm];
+                for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(t16[t]);
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                for (int i = 0; i < kIssuers; ++i) mbar_arrive(&dempty[2 * i + db]);
-            named_bar(1, 128);
+            const int ch = chan_of_row(32 * quad + lane);
+#pragma unroll
+            for (int t = 0; t < 16; ++t) zsm[(tok0 + t) * 128 + ch] = acc[t];
+        }
+        tc_fence_before();
+        named_bar(1, 32 * kDec);
+
+        // ---- a block split over several CTAs: the last to arrive finishes it ----
+        bool finish = true;
+        if (nseg < C) {
             const int p_first = cta_of_unit((long long)g * C, prm.P, prm.U);
             const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
-            bool finish = true;
-            if (p_last > p_first) {
+            {
                 float4* myslot = reinterpret_cast<float4*>(prm.part + (size_t)(p + g) * NT * 128);
                 const float4* z4s = reinterpret_cast<const float4*>(zsm);
-                for (int f = et; f < a.m * 32; f += 128) __stcg(myslot + f, z4s[f]);
+                for (int f = threadIdx.x; f < a.m * 32; f += 32 * kDec) __stcg(myslot + f, z4s[f]);
                 __threadfence();
-                named_bar(1, 128);
-                if (et == 0) {
-                    const uint32_t prev = atomicAdd(&prm.counters[g], 1u);
-                    misc[2] = (prev == (uint32_t)(p_last - p_first)) ? 1 : 0;
-                }
-                named_bar(1, 128);
-                finish = misc[2] != 0;
-                if (finish) {
-                    __threadfence();
-                    reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, et, zsm);
-                    if (et == 0) prm.counters[g] = 0u;
-                    named_bar(1, 128);
-                }
             }
+            named_bar(1, 32 * kDec);
+            if (threadIdx.x == 0) {
+                const uint32_t prev = atomicAdd(&prm.counters[g], 1u);
+                misc[2] = (prev == (uint32_t)(p_last - p_first)) ? 1 : 0;
+            }
+            named_bar(1, 32 * kDec);
+            finish = misc[2] != 0;
             if (finish) {
-                // final epilogue for block g: scale, output rotation, signs, store
-                for (int mm = ew; mm < a.m; mm += kEpiWarps) {
-                    const int n0 = 128 * g + 4 * lane;
-                    const float4 z4 = *reinterpret_cast<const float4*>(zsm + mm * 128 + 4 * lane);
-                    const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
-                    const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
-                    const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
-                    const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
-                    const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
-                    const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
-                    float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
-                    fwht128_warp(vv);
-                    vv[0] *= kInvSqrt128 * sg0.x;
-                    vv[1] *= kInvSqrt128 * sg0.y;
-                    vv[2] *= kInvSqrt128 * sg1.x;
-                    vv[3] *= kInvSqrt128 * sg1.y;
-                    const size_t yo = (size_t)mm * a.n_out + n0;
-                    if (a.y_fp32) {
-                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) =
-                            make_float4(vv[0], vv[1], vv[2], vv[3]);
-                    } else {
-                        __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
-                        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) =
-                            *reinterpret_cast<uint2*>(hh);
-                    }
+                __threadfence();
+                reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, threadIdx.x, zsm);
+                if (threadIdx.x == 0) prm.counters[g] = 0u;      // ready for the next call on this stream
+                named_bar(1, 32 * kDec);
+            }
+        }
+        if (finish) {
+            // final epilogue for block g: scale, output rotation, signs, store
+            for (int mm = warp; mm < a.m; mm += kDec) {
+                const int n0 = 128 * g + 4 * lane;
+                const float4 z4 = *reinterpret_cast<const float4*>(zsm + mm * 128 + 4 * lane);
+                const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
+                const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
+                const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+                const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+                const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+                const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+                float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
+                fwht128_warp(vv);
+                vv[0] *= kInvSqrt128 * sg0.x;
+                vv[1] *= kInvSqrt128 * sg0.y;
+                vv[2] *= kInvSqrt128 * sg1.x;
+                vv[3] *= kInvSqrt128 * sg1.y;
+                const size_t yo = (size_t)mm * a.n_out + n0;
+                if (a.y_fp32) {
+                    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) =
+                        make_float4(vv[0], vv[1], vv[2], vv[3]);
+                } else {
+                    __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
+                    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) = *reinterpret_cast<uint2*>(hh);
                 }
             }
-            named_bar(1, 128);
-            ++seg;
-            u0 += len;
-            c0 = 0;
-            ++g;
         }
-    } else {
-        // ------------------------------------------------------ decoders ---
-        const int d = warp - kWarpDec0;           // 0..15
-        const int slot = d >> 2;                  // units u = slot (mod 4); tile row d % 4 of each
-        const int j = lane >> 2, q = lane & 3;
-        const int src_prev = (lane & ~3) | ((q + 3) & 3);
-        uint32_t soff[2][2];
-        {
-            const int atom = j >> 2, j4 = j & 3;
-#pragma unroll
-            for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
-        }
-        const uint8_t* ring = smem + L::off_p + (size_t)d * kRing * L::ROWB;
-        const uint32_t ast0 = smem_u32(smem + L::off_a + d * kABytes);  // stage d (+ kDecWarps for buffer 1)
-        const int nk = n > slot ? (n - slot + 3) / 4 : 0;      // units this decoder handles
-        for (int k = 0; k < nk; ++k) {
-            const int rs = k % kRing;
-            if (!warp_wait(&pfull[d * kRing + rs], (k / kRing) & 1, abort_flag, kSleepNs)) break;
-            const uint32_t* sw = reinterpret_cast<const uint32_t*>(ring + rs * L::ROWB) + j * TW + q * QW;
-            uint32_t buf[QW + 1];
-            if constexpr (QW % 4 == 0) {
-#pragma unroll
-                for (int w = 0; w < QW / 4; ++w) {
-                    const uint4 vv = reinterpret_cast<const uint4*>(sw)[w];
-                    buf[1 + 4 * w] = vv.x; buf[2 + 4 * w] = vv.y; buf[3 + 4 * w] = vv.z; buf[4 + 4 * w] = vv.w;
-                }
-            } else {
-#pragma unroll
-                for (int w = 0; w < QW / 2; ++w) {
-                    const uint2 vv = reinterpret_cast<const uint2*>(sw)[w];
-                    buf[1 + 2 * w] = vv.x; buf[2 + 2 * w] = vv.y;
-                }
-            }
-            buf[0] = __shfl_sync(0xffffffffu, buf[QW], src_prev);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&pempty[d * kRing + rs]);      // slot free for the producer
-            const int ab = k & 1;
-            if (!warp_wait(&aempty[slot * kABuf + ab], ((k >> 1) & 1) ^ 1, abort_flag, kSleepNs)) break;
-            decode_quarter_to_a<BITS>(buf, ast0 + ab * kDecWarps * kABytes, soff);
-            fence_proxy_async_smem();
-            // the unit's xt chunk must have landed before its MMAs are issued;
-            // the decoder checks it here so that the issuer waits only on afull
-            if (!warp_wait(&bfull[slot * kSB + k % kSB], (k / kSB) & 1, abort_flag, kSleepNs)) break;
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&afull[slot * kABuf + ab]);
-        }
+        named_bar(1, 32 * kDec);                            // zsm and the accumulators free for the next segment
+        tc_fence_after();
+        u0 = u1;
+    }
     }
 
     // ------------------------------------------------------------ teardown ---
     tc_fence_before();
     __syncthreads();
-    if (warp == kWarpIss0) {
+    if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
     }
@@ -552,20 +488,23 @@ __global__ void __launch_bounds__(256) xt_prepass_kernel(const __half* __restric
 
 int nt_for(int m) { return m <= 16 ? 16 : 32; }
 
+size_t xt_offset(int G) { return align_up(ws_counter_off() + 4 * (size_t)G, 1024); }
+
 template <int BITS, int NT>
 cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
 {
-    using L = TcLayout<BITS, NT>;
+    using L = TcLayout<NT>;
     TcParams prm;
     prm.a = a;
     prm.G = a.n_out / 128;
-    prm.C = a.k_in / 64;
+    prm.C = a.k_in / 128;
     prm.U = (long long)prm.G * prm.C;
     prm.P = tc_ctas(a.m, a.k_in, a.n_out, a.bits);
+    prm.two16 = 0x10000u;
     uint8_t* ws = a.ws;
     prm.status = reinterpret_cast<uint32_t*>(ws);
     prm.counters = reinterpret_cast<uint32_t*>(ws + ws_counter_off());
-    const size_t xt_off = align_up(ws_counter_off() + 4 * (size_t)prm.G, 1024);
+    const size_t xt_off = xt_offset(prm.G);
     prm.xt = ws + xt_off;
     prm.part = reinterpret_cast<float*>(ws + align_up(xt_off + (size_t)a.k_in * NT * 2, 256));
 
@@ -592,9 +531,12 @@ int tc_ctas(int m, int k_in, int n_out, int bits)
 {
     (void)m;
     (void)bits;
-    const long long U = (long long)(n_out / 128) * (k_in / 64);
-    long long p = U / kMinUnitsPerCta;
-    if (p > kMaxCtas) p = kMaxCtas;
+    const long long U = (long long)(n_out / 128) * (k_in / 128);
+    long long p = (long long)kSms * kCtasPerSm;       // one wave, two CTAs per SM
+    // at most 8 CTAs per output block on average: the last CTA of a block
+    // reads every partial of it, so small problems use fewer, longer CTAs
+    if (p > 8LL * (n_out / 128)) p = 8LL * (n_out / 128);
+    if (p > U) p = U;                                 // at least one unit per CTA
     if (p < 1) p = 1;
     return (int)p;
 }
@@ -603,8 +545,7 @@ size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
     const int NT = nt_for(m);
     const int G = n_out / 128;
-    const size_t xt_off = align_up(ws_counter_off() + 4 * (size_t)G, 1024);
-    const size_t part_off = align_up(xt_off + (size_t)k_in * NT * 2, 256);
+    const size_t part_off = align_up(xt_offset(G) + (size_t)k_in * NT * 2, 256);
     return part_off + (size_t)(tc_ctas(m, k_in, n_out, bits) + G) * NT * 128 * sizeof(float);
 }
 

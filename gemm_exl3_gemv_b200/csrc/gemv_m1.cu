@@ -54,56 +54,6 @@ template <int BITS>
 constexpr int kM1MinBlocks = 3;
 constexpr int kSms = 148;
 
-// Isolate the 16-bit window that starts P bits after the most significant bit
-// of buf[0] (P a compile-time constant).  Windows at the top or bottom half
-// of a word take one instruction.  Otherwise ALT selects the form:
-//   ALT = false: shift right + mask (two integer-pipe instructions);
-//   ALT = true : shift left so the window is the top half, then a high
-//                multiply by 2^16 (`two16` is a runtime value, so the
-//                multiply stays on the FMA pipe) -- one integer-pipe and one
-//                FMA-pipe instruction.
-template <int P, int NW, bool ALT>
-__device__ __forceinline__ uint32_t window_of(const uint32_t (&buf)[NW], uint32_t two16)
-{
-    constexpr int wi = P >> 5, off = P & 31;
-    static_assert(wi + (off > 16 ? 1 : 0) < NW, "window outside the buffer");
-    if constexpr (off == 0) {
-        return buf[wi] >> 16;
-    } else if constexpr (off == 16) {
-        return buf[wi] & 0xFFFFu;
-    } else if constexpr (!ALT) {
-        if constexpr (off < 16) return (buf[wi] >> (16 - off)) & 0xFFFFu;
-        else return __funnelshift_r(buf[wi + 1], buf[wi], 48 - off) & 0xFFFFu;
-    } else {
-        uint32_t v;
-        if constexpr (off < 16) v = buf[wi] << off;
-        else v = __funnelshift_l(buf[wi + 1], buf[wi], off);
-        return __umulhi(v, two16);
-    }
-}
-
-// Byte-aligned variant for even bit widths: a window whose offset is r bits
-// (r = off mod 8) past a byte boundary is read from the stream shifted left
-// by r bits (one funnel shift per word, shared by every window of that word
-// with the same r), where it sits at a byte boundary: top half (shift), bytes
-// 1-2 (byte permute with zero fill) or bottom half (mask) -- one instruction.
-// Windows that straddle the next word fall back to window_of.
-template <int P, int NW>
-__device__ __forceinline__ uint32_t window_bytes(const uint32_t (&buf)[NW], uint32_t two16)
-{
-    constexpr int wi = P >> 5, off = P & 31, r = off & 7, ob = off - r;
-    if constexpr (ob == 24 || (r != 0 && wi + 1 >= NW)) {
-        return window_of<P, NW, false>(buf, two16);
-    } else {
-        uint32_t w;
-        if constexpr (r == 0) w = buf[wi];
-        else w = __funnelshift_l(buf[wi + 1], buf[wi], r);
-        if constexpr (ob == 0) return w >> 16;
-        else if constexpr (ob == 8) return __byte_perm(w, 0u, 0x4421);
-        else return w & 0xFFFFu;
-    }
-}
-
 __device__ __forceinline__ __half2 as_h2(uint32_t u)
 {
     return *reinterpret_cast<const __half2*>(&u);
@@ -141,33 +91,6 @@ __device__ __forceinline__ void quarter_hfma(const uint32_t (&buf)[NW], const __
         if constexpr (FIRST && R < 16) acc[R & 15] = __hmul2(as_h2(m), xx[R >> 4]);
         else acc[R & 15] = __hfma2(as_h2(m), xx[R >> 4], acc[R & 15]);
         quarter_hfma<BITS, R + 1, FIRST, ALT_EVERY>(buf, xx, acc, two16);
-    }
-}
-
-// Lane's words of one tile row: 2*BITS consecutive words at `src`.
-template <int BITS>
-__device__ __forceinline__ void load_quarter(uint32_t (&w)[2 * BITS], const uint32_t* src)
-{
-    if constexpr (BITS == 3) {
-#pragma unroll
-        for (int t = 0; t < 3; ++t) {
-            uint2 v;
-            asm volatile("ld.global.cs.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(src + 2 * t));
-            w[2 * t] = v.x;
-            w[2 * t + 1] = v.y;
-        }
-    } else {
-#pragma unroll
-        for (int t = 0; t < BITS / 2; ++t) {
-            uint4 v;
-            asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "l"(src + 4 * t));
-            w[4 * t] = v.x;
-            w[4 * t + 1] = v.y;
-            w[4 * t + 2] = v.z;
-            w[4 * t + 3] = v.w;
-        }
     }
 }
 
@@ -237,7 +160,7 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         const uint32_t* src =
             a.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
         uint32_t wa[QW], wb[QW];
-        if (nw > 0) load_quarter<BITS>(wa, src);                       // in flight during the rotation
+        if (nw > 0) load_lane_words<BITS>(wa, src);                       // in flight during the rotation
 
         __syncthreads();                                               // previous segment done with smem
         // input rotation of the touched blocks: xxs[k - 128 kb_lo] = (xt, xt)
@@ -269,9 +192,9 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         __half2 acc[16];
         int i = 0;
         for (; i + 2 <= nw; i += 2) {
-            load_quarter<BITS>(wb, src + (size_t)(i + 1) * row_step);
+            load_lane_words<BITS>(wb, src + (size_t)(i + 1) * row_step);
             tile_row<BITS, true, ALT_EVERY>(wa, xxs, kx0 + i * kx_step, src_prev, acc, two16);
-            if (i + 2 < nw) load_quarter<BITS>(wa, src + (size_t)(i + 2) * row_step);
+            if (i + 2 < nw) load_lane_words<BITS>(wa, src + (size_t)(i + 2) * row_step);
             tile_row<BITS, false, ALT_EVERY>(wb, xxs, kx0 + (i + 1) * kx_step, src_prev, acc, two16);
 #pragma unroll
             for (int c = 0; c < 16; ++c) accf[c] = add_pair_f32(accf[c], acc[c]);
