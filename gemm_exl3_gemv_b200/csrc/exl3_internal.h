@@ -28,8 +28,9 @@ struct GemmArgs {
 size_t m1_workspace_bytes(int k_in, int n_out, int bits);
 cudaError_t launch_gemv_m1(const GemmArgs& a, cudaStream_t stream);
 
-// Tensor-core path (2..32 rows): CTA count, workspace size, launcher (two
-// launches per call: input rotation pre-pass and the product kernel).
+// Tensor-core path (2..32 rows): CTA count (planned), workspace size,
+// launcher (two launches per call: input rotation pre-pass and the product
+// kernel, launched as clusters of the CTAs that share an output block).
 int tc_ctas(int m, int k_in, int n_out, int bits);
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);

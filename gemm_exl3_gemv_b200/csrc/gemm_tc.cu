@@ -37,7 +37,10 @@
 //   * Every mbarrier wait is bounded (2 s); on expiry the CTA records a
 //     timeout in the workspace status word and winds down.
 #include <atomic>
+#include <mutex>
 #include <utility>
+
+#include <cooperative_groups.h>
 
 #include "exl3_common.cuh"
 #include "exl3_decode.cuh"
@@ -45,6 +48,8 @@
 #include "exl3_tc.cuh"
 
 namespace exl3 {
+
+namespace cg = cooperative_groups;
 
 namespace {
 
@@ -79,13 +84,24 @@ struct TcLayout {
     static_assert(kCtasPerSm * total <= 227 * 1024, "two CTAs per SM");
 };
 
+// Two ways to cut the G x C units (output block g, 128-row input block c):
+//   cluster (S > 0): S CTAs per output block, launched as one cluster; CTA r
+//     takes units [rC/S, (r+1)C/S) of its block; the S partial sums meet in
+//     distributed shared memory.  Best when few CTAs per block fill the GPU
+//     poorly otherwise, or when many would have to share a block.
+//   stream-K (S == 0): P equal contiguous ranges of the block-major unit
+//     order, one per CTA; partial sums of blocks cut between CTAs go through
+//     the workspace and the last CTA to arrive adds them.  Best balance when
+//     a block is shared by only a few CTAs.
 struct TcParams {
     GemmArgs a;
     const uint8_t* xt;      // rotated input, B-operand layout
-    float* part;            // segment partial sums, [slot][NT][128]
-    uint32_t* counters;     // per output block
+    float* part;            // stream-K partial sums, [slot][NT][128]
+    uint32_t* counters;     // stream-K arrival counters, per output block
     uint32_t* status;       // workspace status word
-    int G, C, P;            // output blocks, 128-row input blocks, CTAs
+    int C;                  // 128-row input blocks (units per output block)
+    int S;                  // cluster size (CTAs per output block), 0: stream-K
+    int P;                  // stream-K CTAs
     long long U;            // units = G * C
     uint32_t two16;         // 2^16, passed at run time (keeps a multiply on the FMA pipe)
 };
@@ -109,24 +125,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
             return false;
         }
     }
-}
-
-// Warp-wide wait: every lane observes the completed phase (acquire per lane).
-__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
-{
-    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
-    int ok = 0;
-    if ((threadIdx.x & 31) == 0) ok = wait_or_abort(bar, parity, abort_flag) ? 1 : 0;
-    ok = __shfl_sync(0xffffffffu, ok, 0);
-    if (!ok) return false;
-    // the phase has completed and cannot advance again before this warp acts
-    // on it, so this succeeds at once; bounded all the same
-    int tries = 0;
-    while (!mbar_try_wait(bar, parity) && ++tries < (1 << 20)) {
-    }
-    ok = __all_sync(0xffffffffu, tries < (1 << 20)) ? 1 : 0;
-    if (!ok && (threadIdx.x & 31) == 0) atomicExch((int*)abort_flag, 1);
-    return ok != 0;
 }
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
@@ -223,6 +221,39 @@ __device__ __forceinline__ void reduce_segments(const float* part, int g, int p_
     }
 }
 
+// Final epilogue of one output row mm of block g, by one warp: z (this lane's
+// channels 4*lane .. +3) times scale, output rotation, signs, store.
+__device__ __forceinline__ void finish_row_regs(const GemmArgs& a, int g, int mm, const float (&z)[4], int lane)
+{
+    const int n0 = 128 * g + 4 * lane;
+    const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
+    const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
+    const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+    const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+    const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+    const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+    float vv[4] = {z[0] * sc0.x, z[1] * sc0.y, z[2] * sc1.x, z[3] * sc1.y};
+    fwht128_warp(vv);
+    vv[0] *= kInvSqrt128 * sg0.x;
+    vv[1] *= kInvSqrt128 * sg0.y;
+    vv[2] *= kInvSqrt128 * sg1.x;
+    vv[3] *= kInvSqrt128 * sg1.y;
+    const size_t yo = (size_t)mm * a.n_out + n0;
+    if (a.y_fp32) {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+    } else {
+        __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
+        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) = *reinterpret_cast<uint2*>(hh);
+    }
+}
+
+__device__ __forceinline__ void finish_row(const GemmArgs& a, int g, int mm, const float* zrow, int lane)
+{
+    const float4 z4 = *reinterpret_cast<const float4*>(zrow + 4 * lane);
+    const float z[4] = {z4.x, z4.y, z4.z, z4.w};
+    finish_row_regs(a, g, mm, z, lane);
+}
+
 template <int BITS, int NT>
 __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParams prm)
 {
@@ -234,18 +265,26 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     uint64_t* aempty = bar;                                   // [kDec][kAStages]: the stage's MMA completed
     uint64_t* bfull = aempty + kDec * kAStages;               // [kBStages]: xt unit landed
     uint64_t* bempty = bfull + kBStages;                      // [kBStages]: all 8 MMAs on it completed
-    uint64_t* segdone = bempty + kBStages;                    // every accumulator of the segment final
-    int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort, [2] last-CTA flag
+    uint64_t* segdone = bempty + kBStages;                    // every accumulator final
+    int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
 
     const GemmArgs& a = prm.a;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int S = prm.S, C = prm.C;
     const int p = blockIdx.x;
-    const long long b0 = (long long)p * prm.U / prm.P;
-    const long long b1 = (long long)(p + 1) * prm.U / prm.P;
-    const int C = prm.C;
     const int tiles_n = a.n_out / 16;
+    // this CTA's units [b0, b1) in block-major order
+    long long b0, b1;
+    if (S > 0) {
+        const int gc = p / S, rc = p % S;
+        b0 = (long long)gc * C + (long long)rc * C / S;
+        b1 = (long long)gc * C + (long long)(rc + 1) * C / S;
+    } else {
+        b0 = (long long)p * prm.U / prm.P;
+        b1 = (long long)(p + 1) * prm.U / prm.P;
+    }
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < kDec * kAStages; ++i) mbar_init(&aempty[i], 1);
@@ -277,58 +316,63 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
                 if (++c == C) c = 0;
             }
-            // let every issued copy land before the CTA can exit
+            // on abort, let every issued copy land before the CTA can exit
             const int issued = kk;
             for (int v = issued > kBStages ? issued - kBStages : 0; v < issued; ++v) {
                 if (*abort_flag)
                     (void)mbar_wait_bounded(&bfull[v & (kBStages - 1)], (uint32_t)(v / kBStages) & 1u, 100000000ull);
             }
         }
-
     } else {
-    // ---- decoder warps: the segment loop (the producer never joins their
-    // barriers, which are the 256-thread named barrier 1) ----
-    const int j = lane >> 2, q = lane & 3;
-    const int src_prev = (lane & ~3) | ((q + 3) & 3);
-    uint32_t soff[2][2];
-    {
-        const int atom = j >> 2, j4 = j & 3;
-#pragma unroll
-        for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-            for (int e = 0; e < 2; ++e)
-                soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
-    }
-    constexpr uint32_t idesc = idesc_f16_amn(128, NT);
-    static_assert(kAStages == 2, "A stage index = unit counter & 1");
-    static_assert((kBStages & (kBStages - 1)) == 0, "power of two");
-    const uint32_t ast0 = smem_u32(smem + L::off_a + (warp * kAStages + 0) * kABytes);
-    const uint32_t ast1 = smem_u32(smem + L::off_a + (warp * kAStages + 1) * kABytes);
-    const uint64_t adesc0 = sdesc_sw128(ast0, 1024, 2048), adesc1 = sdesc_sw128(ast1, 1024, 2048);
-    // this warp's tile row is rows 16*warp .. +15 of the unit: chunk warp/4, 32 bytes per 16 rows
-    const uint32_t bw = (uint32_t)((warp >> 2) * L::CHUNK + (warp & 3) * 32);
-    // stage bs adds bs * BUNIT to the start address (no carry out of the 14-bit field: smem < 256 KB)
-    const uint64_t bdesc0 = sdesc_sw128(smem_u32(smem + L::off_b) + bw, 16, 1024);
-    const uint32_t dcol = tmem + (uint32_t)(warp * NT);
-    int kk = 0;                // unit counter of this CTA (stage and parity index)
-    int seg = 0;
-    for (long long u0 = b0; u0 < b1; ++seg) {
-        const int g = (int)(u0 / C);
-        const int c0 = (int)(u0 - (long long)g * C);
-        const long long u1 = ((long long)(g + 1) * C < b1) ? (long long)(g + 1) * C : b1;
-        const int nseg = (int)(u1 - u0);
-
+        // --------------------------------------------- decoder warps ---
+        // Segment loop: the CTA's units grouped by output block (one segment
+        // in cluster mode).  The producer never joins these warps' barriers
+        // (the 256-thread named barrier 1).
+        const int q = lane & 3;
+        const int src_prev = (lane & ~3) | ((q + 3) & 3);
+        uint32_t soff[2][2];
         {
-            // --------------------------------------------- decoder warp ---
-            const uint32_t* src = a.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
-            const size_t unit_step = (size_t)8 * tiles_n * TW;        // words between consecutive units
-            bool ok = true;
-            // decode unit k (the CTA's kk-th) from `wds` into A stage kk & 1, then
-            // lane 0 issues its MMA into this warp's accumulator
-            auto unit = [&](const uint32_t (&wds)[QW], int k, int kk) {
-                const int s = kk & (kAStages - 1), bs = kk & (kBStages - 1);
-                const uint32_t ph = (uint32_t)(kk / kAStages) & 1u, bph = (uint32_t)(kk / kBStages) & 1u;
-                if (kk >= kAStages && !warp_wait(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag)) ok = false;
+            const int j = lane >> 2, atom = j >> 2, j4 = j & 3;
+#pragma unroll
+            for (int rb = 0; rb < 2; ++rb)
+#pragma unroll
+                for (int e = 0; e < 2; ++e)
+                    soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
+        }
+        constexpr uint32_t idesc = idesc_f16_amn(128, NT);
+        static_assert(kAStages == 2, "A stage index = unit counter & 1");
+        static_assert((kBStages & (kBStages - 1)) == 0, "power of two");
+        const uint32_t ast0 = smem_u32(smem + L::off_a + (warp * kAStages + 0) * kABytes);
+        const uint32_t ast1 = smem_u32(smem + L::off_a + (warp * kAStages + 1) * kABytes);
+        const uint64_t adesc0 = sdesc_sw128(ast0, 1024, 2048), adesc1 = sdesc_sw128(ast1, 1024, 2048);
+        // this warp's tile row is rows 16*warp .. +15 of a unit: chunk warp/4, 32 bytes per 16 rows;
+        // stage bs adds bs * BUNIT to the start address (no carry out of its 14-bit field: smem < 256 KB)
+        const uint32_t bw = (uint32_t)((warp >> 2) * L::CHUNK + (warp & 3) * 32);
+        const uint64_t bdesc0 = sdesc_sw128(smem_u32(smem + L::off_b) + bw, 16, 1024);
+        const uint32_t dcol = tmem + (uint32_t)(warp * NT);
+        bool fail0 = false;                                      // lane 0: a wait gave up
+        int kk = 0;                                              // CTA unit counter (stages, parities)
+        int seg = 0;
+        for (long long u0 = b0; u0 < b1; ++seg) {
+            const int g = (int)(u0 / C);
+            const int c0 = (int)(u0 - (long long)g * C);
+            const long long u1 = ((long long)(g + 1) * C < b1) ? (long long)(g + 1) * C : b1;
+            const int nseg = (int)(u1 - u0);
+            const uint32_t* src =
+                a.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
+            const size_t unit_step = (size_t)8 * tiles_n * TW;    // words between consecutive units
+            bool ok = true;                                      // warp-uniform
+            // decode the segment's unit k (the CTA's kk-th) from `wds` into A
+            // stage kk & 1, then lane 0 issues its MMA into this warp's accumulator
+            auto unit = [&](const uint32_t (&wds)[QW], int k, int kq) {
+                const int s = kq & (kAStages - 1), bs = kq & (kBStages - 1);
+                const uint32_t ph = (uint32_t)(kq / kAStages) & 1u, bph = (uint32_t)(kq / kBStages) & 1u;
+                // lane 0 waits for the MMA that last read this stage; the shuffle
+                // then orders every lane's stores after it
+                int okw = 1;
+                if (lane == 0)
+                    okw = !fail0 && (kq < kAStages || wait_or_abort(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag));
+                if (!__shfl_sync(0xffffffffu, okw, 0)) ok = false;
                 if (!ok) return;
                 uint32_t buf[QW + 1];
                 buf[0] = __shfl_sync(0xffffffffu, wds[QW - 1], src_prev);
@@ -337,14 +381,17 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 decode_quarter_to_a<BITS>(buf, s ? ast1 : ast0, soff, prm.two16);
                 fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
-                if (lane == 0 && wait_or_abort(&bfull[bs], bph, abort_flag)) {
-                    tc_fence_after();
-                    const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);   // start address field
-                    mma_f16_ss(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
-                    mma_commit(&aempty[warp * kAStages + s]);
-                    mma_commit(&bempty[bs]);
+                if (lane == 0) {
+                    if (wait_or_abort(&bfull[bs], bph, abort_flag)) {
+                        tc_fence_after();
+                        const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
+                        mma_f16_ss(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
+                        mma_commit(&aempty[warp * kAStages + s]);
+                        mma_commit(&bempty[bs]);
+                    } else {
+                        fail0 = true;                    // seen by the whole warp at its next unit
+                    }
                 }
-                ok = __shfl_sync(0xffffffffu, *abort_flag == 0 ? 1 : 0, 0) != 0;
             };
             uint32_t wa[QW], wb[QW];
             load_lane_words<BITS>(wa, src);
@@ -357,93 +404,103 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             }
             if (k < nseg) unit(wa, k, kk + k);
             kk += nseg;
+            ok = __shfl_sync(0xffffffffu, (ok && !fail0) ? 1 : 0, 0) != 0;
             if (lane == 0) {
                 if (ok) mma_commit(segdone);             // arrives once this warp's MMAs are done
                 else mbar_arrive(segdone);
             }
-        }
 
-        // ---- segment epilogue: accumulators -> zsm[NT][128] ----
-        bool ok = warp_wait(segdone, (uint32_t)(seg & 1), abort_flag);
-        tc_fence_after();
-        constexpr int kReaders = NT == 32 ? 8 : 4;         // warps reading the accumulators
-        if (warp < kReaders && ok) {
-            const int quad = warp & 3;                       // tensor-memory lanes 32*quad .. +31
-            const int tok0 = (warp >> 2) * 16;               // 16 rows (accumulator columns) per warp
-            float acc[16];
+            // ---- accumulators -> zsm[NT][128] (the eight summed in a fixed order) ----
+            int okd = 1;
+            if (lane == 0) okd = wait_or_abort(segdone, (uint32_t)(seg & 1), abort_flag) ? 1 : 0;
+            okd = __shfl_sync(0xffffffffu, okd, 0);
+            tc_fence_after();
+            constexpr int kReaders = NT == 32 ? 8 : 4;     // warps reading the accumulators
+            if (warp < kReaders) {
+                const int quad = warp & 3;                   // tensor-memory lanes 32*quad .. +31
+                const int tok0 = (warp >> 2) * 16;           // 16 rows (accumulator columns) per warp
+                float acc[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+                for (int t = 0; t < 16; ++t) acc[t] = 0.f;
+                if (okd) {
 #pragma unroll
-            for (int w = 0; w < kDec; ++w) {
-                uint32_t t16[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(w * NT + tok0), t16);
-                tmem_ld_wait();
+                    for (int w = 0; w < kDec; ++w) {
+                        uint32_t t16[16];
+                        tmem_ld16(tmem + ((uint32_t)(32 * quad) << 16) + (uint32_t)(w * NT + tok0), t16);
+                        tmem_ld_wait();
 #pragma unroll
-                for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(t16[t]);
+                        for (int t = 0; t < 16; ++t) acc[t] += __uint_as_float(t16[t]);
+                    }
+                }
+                const int ch = chan_of_row(32 * quad + lane);
+#pragma unroll
+                for (int t = 0; t < 16; ++t) zsm[(tok0 + t) * 128 + ch] = acc[t];
             }
-            const int ch = chan_of_row(32 * quad + lane);
-#pragma unroll
-            for (int t = 0; t < 16; ++t) zsm[(tok0 + t) * 128 + ch] = acc[t];
-        }
-        tc_fence_before();
-        named_bar(1, 32 * kDec);
+            tc_fence_before();
+            if (S > 0) break;                                // cluster mode: one segment, finished below
 
-        // ---- a block split over several CTAs: the last to arrive finishes it ----
-        bool finish = true;
-        if (nseg < C) {
-            const int p_first = cta_of_unit((long long)g * C, prm.P, prm.U);
-            const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
-            {
+            // ---- stream-K: a block cut over several CTAs, the last to arrive finishes it ----
+            named_bar(1, 32 * kDec);
+            bool finish = true;
+            if (nseg < C) {
+                const int p_first = cta_of_unit((long long)g * C, prm.P, prm.U);
+                const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
                 float4* myslot = reinterpret_cast<float4*>(prm.part + (size_t)(p + g) * NT * 128);
                 const float4* z4s = reinterpret_cast<const float4*>(zsm);
                 for (int f = threadIdx.x; f < a.m * 32; f += 32 * kDec) __stcg(myslot + f, z4s[f]);
                 __threadfence();
-            }
-            named_bar(1, 32 * kDec);
-            if (threadIdx.x == 0) {
-                const uint32_t prev = atomicAdd(&prm.counters[g], 1u);
-                misc[2] = (prev == (uint32_t)(p_last - p_first)) ? 1 : 0;
-            }
-            named_bar(1, 32 * kDec);
-            finish = misc[2] != 0;
-            if (finish) {
-                __threadfence();
-                reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, threadIdx.x, zsm);
-                if (threadIdx.x == 0) prm.counters[g] = 0u;      // ready for the next call on this stream
                 named_bar(1, 32 * kDec);
-            }
-        }
-        if (finish) {
-            // final epilogue for block g: scale, output rotation, signs, store
-            for (int mm = warp; mm < a.m; mm += kDec) {
-                const int n0 = 128 * g + 4 * lane;
-                const float4 z4 = *reinterpret_cast<const float4*>(zsm + mm * 128 + 4 * lane);
-                const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
-                const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
-                const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
-                const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
-                const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
-                const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
-                float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
-                fwht128_warp(vv);
-                vv[0] *= kInvSqrt128 * sg0.x;
-                vv[1] *= kInvSqrt128 * sg0.y;
-                vv[2] *= kInvSqrt128 * sg1.x;
-                vv[3] *= kInvSqrt128 * sg1.y;
-                const size_t yo = (size_t)mm * a.n_out + n0;
-                if (a.y_fp32) {
-                    *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) =
-                        make_float4(vv[0], vv[1], vv[2], vv[3]);
-                } else {
-                    __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
-                    *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) = *reinterpret_cast<uint2*>(hh);
+                if (threadIdx.x == 0) {
+                    const uint32_t prev = atomicAdd(&prm.counters[g], 1u);
+                    misc[2] = (prev == (uint32_t)(p_last - p_first)) ? 1 : 0;
+                }
+                named_bar(1, 32 * kDec);
+                finish = misc[2] != 0;
+                if (finish) {
+                    __threadfence();
+                    reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, threadIdx.x, zsm);
+                    if (threadIdx.x == 0) prm.counters[g] = 0u;      // ready for the next call on this stream
+                    named_bar(1, 32 * kDec);
                 }
             }
+            if (finish)
+                for (int mm = warp; mm < a.m; mm += kDec) finish_row(a, g, mm, zsm + mm * 128, lane);
+            named_bar(1, 32 * kDec);                         // zsm and the accumulators free for the next segment
+            tc_fence_after();
+            u0 = u1;
         }
-        named_bar(1, 32 * kDec);                            // zsm and the accumulators free for the next segment
-        tc_fence_after();
-        u0 = u1;
     }
+
+    // ---- cluster mode: the cluster's CTAs add their z in rank order
+    // (distributed shared memory) and each finishes every S-th row ----
+    if (S > 0) {
+        cg::cluster_group cluster = cg::this_cluster();
+        const int g = p / S, r = p % S;
+        cluster.sync();                                      // every z of the cluster written
+        if (warp < kDec) {
+            for (int mm = r + S * warp; mm < a.m; mm += S * kDec) {
+                // all S loads in flight first, then added in rank order
+                float4 v[16];
+#pragma unroll
+                for (int qr = 0; qr < 16; ++qr) {
+                    v[qr] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (qr < S) {
+                        const float* peer = cluster.map_shared_rank(zsm, qr);
+                        v[qr] = *reinterpret_cast<const float4*>(peer + mm * 128 + 4 * lane);
+                    }
+                }
+                float4 z4 = v[0];
+#pragma unroll
+                for (int qr = 1; qr < 16; ++qr) {
+                    if (qr < S) {
+                        z4.x += v[qr].x; z4.y += v[qr].y; z4.z += v[qr].z; z4.w += v[qr].w;
+                    }
+                }
+                float zr[4] = {z4.x, z4.y, z4.z, z4.w};
+                finish_row_regs(a, g, mm, zr, lane);
+            }
+        }
+        cluster.sync();                                      // no CTA leaves while its z is being read
     }
 
     // ------------------------------------------------------------ teardown ---
@@ -490,23 +547,92 @@ int nt_for(int m) { return m <= 16 ? 16 : 32; }
 
 size_t xt_offset(int G) { return align_up(ws_counter_off() + 4 * (size_t)G, 1024); }
 
+// stream-K CTA count: one wave (two CTAs per SM), at most 8 CTAs per output
+// block on average (the last CTA of a block reads every partial of it), at
+// most one CTA per unit
+int sk_ctas(int k_in, int n_out)
+{
+    const long long G = n_out / 128, U = G * (k_in / 128);
+    long long p = (long long)kSms * kCtasPerSm;
+    if (p > 8 * G) p = 8 * G;
+    if (p > U) p = U;
+    if (p < 1) p = 1;
+    return (int)p;
+}
+
+size_t part_offset(int k_in, int n_out, int NT) { return align_up(xt_offset(n_out / 128) + (size_t)k_in * NT * 2, 256); }
+
+// Stand-in with the product kernel's block size and shared memory but
+// nothing else, for the cluster-occupancy query: for the product kernel
+// itself (which uses tensor memory) the query reports one CTA per SM,
+// although two run (its registers, threads and shared memory fit twice).
+__global__ void __launch_bounds__(kTcThreads) cluster_fit_probe_kernel(int* never)
+{
+    extern __shared__ int probe_smem[];
+    if (never) never[0] = probe_smem[threadIdx.x];
+}
+
+struct TcPlan {
+    int S;   // > 0: cluster mode with S CTAs per block; 0: stream-K
+    int P;   // CTAs launched
+};
+
+// Pick the cut of the units for this shape: cost in unit-decode times of the
+// busiest CTA, plus the reduction (stream-K: the last CTA reads every partial
+// of its block, about 0.3 unit-times each; cluster: one pass over shared
+// memory).  A cluster size is used only if all G clusters fit at once.
+TcPlan choose_plan(int k_in, int n_out, size_t smem)
+{
+    auto kern = cluster_fit_probe_kernel;
+    const int G = n_out / 128, C = k_in / 128;
+    const long long U = (long long)G * C;
+    TcPlan sk{0, sk_ctas(k_in, n_out)};
+    const double cost_sk = (double)((U + sk.P - 1) / sk.P) + 0.3 * (double)sk.P / G;
+    int Smax = (kSms * kCtasPerSm) / G;
+    if (Smax > 10) Smax = 10;          // measured: 16-CTA clusters were slower than 10 (k/v shapes)
+    if (Smax > C) Smax = C;
+    for (int S = Smax; S >= 1; --S) {
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = S;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(G * S), 1, 1);
+        cfg.blockDim = dim3(kTcThreads, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int nclusters = 0;
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kern, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();
+            continue;
+        }
+        if (nclusters >= G) {
+            const double cost_cl = (double)((C + S - 1) / S) + 0.2 + 0.05 * S;
+            if (cost_cl < cost_sk) return TcPlan{S, G * S};
+            break;
+        }
+    }
+    return sk;
+}
+
 template <int BITS, int NT>
 cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
 {
     using L = TcLayout<NT>;
     TcParams prm;
     prm.a = a;
-    prm.G = a.n_out / 128;
+    const int G = a.n_out / 128;
     prm.C = a.k_in / 128;
-    prm.U = (long long)prm.G * prm.C;
-    prm.P = tc_ctas(a.m, a.k_in, a.n_out, a.bits);
+    prm.U = (long long)G * prm.C;
     prm.two16 = 0x10000u;
     uint8_t* ws = a.ws;
     prm.status = reinterpret_cast<uint32_t*>(ws);
     prm.counters = reinterpret_cast<uint32_t*>(ws + ws_counter_off());
-    const size_t xt_off = xt_offset(prm.G);
+    const size_t xt_off = xt_offset(G);
     prm.xt = ws + xt_off;
-    prm.part = reinterpret_cast<float*>(ws + align_up(xt_off + (size_t)a.k_in * NT * 2, 256));
+    prm.part = reinterpret_cast<float*>(ws + part_offset(a.k_in, a.n_out, NT));
 
     const long long items = (long long)NT * (a.k_in / 128);
     xt_prepass_kernel<NT><<<(unsigned)((items + 7) / 8), 256, 0, stream>>>(
@@ -515,13 +641,55 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     if (e != cudaSuccess) return e;
 
     auto kern = gemm_tc_kernel<BITS, NT>;
-    static std::atomic<int> configured{0};
-    if (!configured.load()) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
-        if (e != cudaSuccess) return e;
-        configured.store(1);
+    static std::once_flag once;
+    static cudaError_t setup = cudaSuccess;
+    std::call_once(once, [&] {
+        setup = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
+        if (setup == cudaSuccess) setup = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (setup == cudaSuccess)
+            setup = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         TcLayout<32>::total);
+        if (setup == cudaSuccess)
+            setup = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    });
+    if (setup != cudaSuccess) return setup;
+
+    // plan decided once per shape (host-side occupancy queries), then cached
+    static std::mutex mu;
+    static long long cache_key[32] = {};
+    static TcPlan cache_val[32];
+    static int cache_next = 0;
+    const long long key = (long long)a.k_in * 1000003LL + a.n_out;
+    TcPlan pl{-1, 0};
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < 32; ++i)
+            if (cache_key[i] == key) pl = cache_val[i];
     }
-    kern<<<prm.P, kTcThreads, L::total, stream>>>(prm);
+    if (pl.S < 0) {
+        pl = choose_plan(a.k_in, a.n_out, L::total);
+        std::lock_guard<std::mutex> lock(mu);
+        cache_key[cache_next] = key;
+        cache_val[cache_next] = pl;
+        cache_next = (cache_next + 1) % 32;
+    }
+    prm.S = pl.S;
+    prm.P = pl.S > 0 ? 0 : pl.P;
+
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.S > 0 ? pl.S : 1;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)pl.P, 1, 1);
+    cfg.blockDim = dim3(kTcThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::total;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, prm);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
@@ -531,22 +699,15 @@ int tc_ctas(int m, int k_in, int n_out, int bits)
 {
     (void)m;
     (void)bits;
-    const long long U = (long long)(n_out / 128) * (k_in / 128);
-    long long p = (long long)kSms * kCtasPerSm;       // one wave, two CTAs per SM
-    // at most 8 CTAs per output block on average: the last CTA of a block
-    // reads every partial of it, so small problems use fewer, longer CTAs
-    if (p > 8LL * (n_out / 128)) p = 8LL * (n_out / 128);
-    if (p > U) p = U;                                 // at least one unit per CTA
-    if (p < 1) p = 1;
-    return (int)p;
+    return sk_ctas(k_in, n_out);
 }
 
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
+    (void)bits;
     const int NT = nt_for(m);
-    const int G = n_out / 128;
-    const size_t part_off = align_up(xt_offset(G) + (size_t)k_in * NT * 2, 256);
-    return part_off + (size_t)(tc_ctas(m, k_in, n_out, bits) + G) * NT * 128 * sizeof(float);
+    // the stream-K partial slots are always reserved (either cut may be chosen)
+    return part_offset(k_in, n_out, NT) + (size_t)(sk_ctas(k_in, n_out) + n_out / 128) * NT * 128 * sizeof(float);
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream)
