@@ -40,7 +40,7 @@ WORKLOAD = "64-layer 27B-class stack (q/k/v/o 5120x5120, 5120x1024 x2, gate/up 5
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--m", type=int, default=32)
@@ -57,6 +57,33 @@ def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+KERNEL_SOURCES = ["gemm_exl3_gemv_b200/csrc/gemm_tc.cu", "gemm_exl3_gemv_b200/csrc/exl3_decode.cuh",
+                  "gemm_exl3_gemv_b200/csrc/exl3_common.cuh", "gemm_exl3_gemv_b200/csrc/exl3_tc.cuh"]
+
+
+def kernel_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic_ratio():
+    """DRAM bytes per packed-weight byte of the verify-GEMM kernel, from the
+    committed ncu capture in profiles/ -- only if the kernel's sources are the
+    ones that capture measured (else None)."""
+    p = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        d = json.load(f)
+    if d.get("source_sha256") != kernel_source_hash():
+        return None, None
+    return float(d["dram_bytes_per_packed_byte"]), d.get("capture")
 
 
 def load_peaks():
@@ -289,6 +316,7 @@ def run_ours(args, world, rank, local):
         sampler = ClockSampler(gpu_id) if m == args.m else None
         if sampler:
             sampler.start()
+            time.sleep(0.5)                             # let nvidia-smi start sampling
         ms = timed(torch, fn, args.steps, args.warmup, barrier)
         clocks = sampler.stop() if sampler else None
         ms = max_over_ranks(ms)
@@ -310,6 +338,8 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = load_peaks()
     algo_bytes = st.packed_bytes + st.io_bytes
     achieved = algo_bytes / (main["ms"] * 1e-3) / 1e9
+    ratio, traffic_src = measured_traffic_ratio() if args.m > 1 else (None, None)
+    traffic = round(ratio * st.packed_bytes / len(st.specs)) if ratio else None
     line = {
         "metric": METRIC, "value": round(gbs * world, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms"], 4),
@@ -327,8 +357,12 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(world * st.packed_bytes / (main["e2e_ms"] * 1e-3) / 1e9, 3), "unit": UNIT,
                 "h2d_bytes_per_step": st.h2d, "d2h_bytes_per_step": st.d2h},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_kind": peak_kind, "kernel": "exl3 product kernel, avg over the step's launches",
+                     "frac": round(achieved / peak, 4), "traffic": traffic,
+                     "peak_kind": peak_kind,
+                     "kernel": "verify product (input-rotation pre-pass + gemm_tc_kernel), per product: "
+                               "algorithmic bytes / (CUDA-event step time / products)",
+                     "algorithmic_bytes_per_product": round(algo_bytes / len(st.specs)),
+                     "traffic_source": traffic_src,
                      "launches_per_step": st.launches},
     }
     if 1 in results and args.m != 1:
