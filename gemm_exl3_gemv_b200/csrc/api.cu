@@ -72,6 +72,7 @@ int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* s
     a.n_out = n_out;
     a.bits = bits;
     a.ws = static_cast<unsigned char*>(ws);
+    a.pdl = 1;
     cudaError_t e = m == 1 ? exl3::launch_gemv_m1(a, static_cast<cudaStream_t>(stream))
                            : exl3::launch_gemm_tc(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
@@ -243,6 +244,7 @@ extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, cons
     a.n_out = n_out;
     a.bits = bits;
     a.ws = static_cast<unsigned char*>(ws);
+    a.pdl = 0;                       // follows a memset: ordinary stream order
     e = exl3::launch_gemv_m1(a, s);
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }

@@ -114,6 +114,16 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
         : "memory");
 }
 
+// ------------------------------------------- programmatic dependent launch ---
+// A kernel launched with programmatic stream serialization may start while
+// the previous kernel of its stream is still running.  grid_dep_wait():
+// block until that kernel has completed and its writes are visible (returns
+// at once for an ordinary launch); every thread that touches memory the
+// previous kernel may read or write calls it first.  grid_dep_launch(): let
+// the next kernel of the stream begin launching its CTAs.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------ Hadamard ---
 // Unnormalised Walsh-Hadamard transform of one 128-element block held by a
 // warp, 4 consecutive elements per lane (element 4*lane + e in v[e]).  Natural

@@ -22,6 +22,7 @@ struct GemmArgs {
     int y_fp32;
     int m, k_in, n_out, bits;
     unsigned char* ws;        // workspace base
+    int pdl;                  // launch with programmatic dependent launch (overlap the previous kernel's tail)
 };
 
 // Single-row product on CUDA cores (gemv_m1.cu).

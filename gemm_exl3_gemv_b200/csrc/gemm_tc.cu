@@ -302,8 +302,10 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = (uint32_t)misc[0];
+    grid_dep_launch();                 // the next kernel may start launching
 
     if (warp == kProdWarp) {
+        grid_dep_wait();               // xt is written by the pre-pass
         // ------------------------------------------------- xt producer ---
         // xt of unit (g, c) is chunks 2c, 2c+1: BUNIT contiguous bytes.
         if (lane == 0) {
@@ -395,6 +397,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             };
             uint32_t wa[QW], wb[QW];
             load_lane_words<BITS>(wa, src);
+            if (seg == 0) grid_dep_wait();     // weights are never written; y and the workspace after this
             int k = 0;
             for (; k + 2 <= nseg; k += 2) {
                 load_lane_words<BITS>(wb, src + (size_t)(k + 1) * unit_step);
@@ -522,6 +525,8 @@ __global__ void __launch_bounds__(256) xt_prepass_kernel(const __half* __restric
                                                          int m_rows, int k_in, uint8_t* __restrict__ xt)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    grid_dep_launch();                 // the product kernel may start its prologue
+    grid_dep_wait();                   // x and the workspace only after the previous kernel
     const int nblk = k_in / 128;
     const long long item = (long long)blockIdx.x * 8 + warp;
     if (item >= (long long)NT * nblk) return;
@@ -635,8 +640,20 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     prm.part = reinterpret_cast<float*>(ws + part_offset(a.k_in, a.n_out, NT));
 
     const long long items = (long long)NT * (a.k_in / 128);
-    xt_prepass_kernel<NT><<<(unsigned)((items + 7) / 8), 256, 0, stream>>>(
-        reinterpret_cast<const __half*>(a.x), reinterpret_cast<const __half*>(a.su), a.m, a.k_in, ws + xt_off);
+    cudaLaunchAttribute pdl_attr;
+    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
+    {
+        cudaLaunchConfig_t pcfg = {};
+        pcfg.gridDim = dim3((unsigned)((items + 7) / 8), 1, 1);
+        pcfg.blockDim = dim3(256, 1, 1);
+        pcfg.stream = stream;
+        pcfg.attrs = &pdl_attr;
+        pcfg.numAttrs = a.pdl ? 1 : 0;
+        cudaError_t e = cudaLaunchKernelEx(&pcfg, xt_prepass_kernel<NT>, reinterpret_cast<const __half*>(a.x),
+                                           reinterpret_cast<const __half*>(a.su), a.m, a.k_in, ws + xt_off);
+        if (e != cudaSuccess) return e;
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -677,17 +694,18 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     prm.P = pl.S > 0 ? 0 : pl.P;
 
     cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = pl.S > 0 ? pl.S : 1;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr;
     cfg.gridDim = dim3((unsigned)pl.P, 1, 1);
     cfg.blockDim = dim3(kTcThreads, 1, 1);
     cfg.dynamicSmemBytes = L::total;
     cfg.stream = stream;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = a.pdl ? 2 : 1;
     e = cudaLaunchKernelEx(&cfg, kern, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();

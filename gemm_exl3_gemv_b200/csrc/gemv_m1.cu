@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     const size_t row_step = (size_t)kM1Warps * tiles_n * TW;          // words between a warp's rows
     float* part = reinterpret_cast<float*>(a.ws + ws_part_off(a.n_out));
     uint32_t* counters = reinterpret_cast<uint32_t*>(a.ws + ws_counter_off());
+    grid_dep_launch();                     // the next product may start loading its weights
+    bool first_seg = true;
 
     for (long long u = b0; u < b1;) {
         // ---- segment: block g, tile rows [r0, r1) ----
@@ -161,6 +163,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
             a.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
         uint32_t wa[QW], wb[QW];
         if (nw > 0) load_lane_words<BITS>(wa, src);                       // in flight during the rotation
+        if (first_seg) grid_dep_wait();    // weights are never written; x, y, workspace only after this
+        first_seg = false;
 
         __syncthreads();                                               // previous segment done with smem
         // input rotation of the touched blocks: xxs[k - 128 kb_lo] = (xt, xt)
@@ -344,7 +348,18 @@ cudaError_t launch_m1_t(const GemmArgs& a, cudaStream_t stream)
         if (e != cudaSuccess) return e;
         configured.store(lim);
     }
-    kern<<<pl.P, kM1Threads, smem, stream>>>(a, pl, 0x10000u);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)pl.P, 1, 1);
+    cfg.blockDim = dim3(kM1Threads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = a.pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a, pl, 0x10000u);
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
 
