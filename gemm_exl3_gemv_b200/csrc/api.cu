@@ -51,6 +51,26 @@ int validate_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16
     return EXL3_OK;
 }
 
+// Problem description of a single product (a group of one sibling).
+exl3::GemmArgs single_args(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale,
+                           const uint16_t* su, const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out,
+                           int bits, void* ws)
+{
+    exl3::GemmArgs a = {};
+    a.x = x;
+    a.su = su;
+    a.y_fp32 = y_fp32 ? 1 : 0;
+    a.m = m;
+    a.k_in = k_in;
+    a.bits = bits;
+    a.n_out = n_out;
+    a.nsib = 1;
+    a.sib[0] = exl3::Sibling{packed, scale, sv, y, n_out, 0};
+    a.ws = static_cast<unsigned char*>(ws);
+    a.pdl = 1;
+    return a;
+}
+
 int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale, const uint16_t* su,
              const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out, int bits, void* ws, size_t ws_bytes,
              void* stream)
@@ -59,20 +79,7 @@ int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* s
     if (st != EXL3_OK) return st;
     st = check_arch();
     if (st != EXL3_OK) return st;
-    exl3::GemmArgs a;
-    a.x = x;
-    a.packed = packed;
-    a.scale = scale;
-    a.su = su;
-    a.sv = sv;
-    a.y = y;
-    a.y_fp32 = y_fp32 ? 1 : 0;
-    a.m = m;
-    a.k_in = k_in;
-    a.n_out = n_out;
-    a.bits = bits;
-    a.ws = static_cast<unsigned char*>(ws);
-    a.pdl = 1;
+    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws);
     cudaError_t e = m == 1 ? exl3::launch_gemv_m1(a, static_cast<cudaStream_t>(stream))
                            : exl3::launch_gemm_tc(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
@@ -169,6 +176,49 @@ int exl3_gemm_small_m(int m, const uint16_t* x, const uint32_t* packed, const ui
 
 }  // extern "C"
 
+// ------------------------------------------------------------- siblings ---
+
+extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, const exl3_matrix_t* mats,
+                                  int n_mats, int y_fp32, int k_in, int bits, void* workspace, size_t ws_bytes,
+                                  void* stream)
+{
+    if (!x || !su || !mats) return EXL3_ERR_INVALID_ARG;
+    if (m <= 0 || k_in <= 0 || n_mats <= 0) return EXL3_ERR_INVALID_ARG;
+    if (n_mats > exl3::kMaxSiblings || m > 32 || !bits_ok(bits) || k_in % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(su)) return EXL3_ERR_MISALIGNED;
+    exl3::GemmArgs a = {};
+    long long total = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const exl3_matrix_t& t = mats[i];
+        if (!t.packed || !t.scale || !t.sv || !t.y) return EXL3_ERR_INVALID_ARG;
+        if (t.n_out <= 0) return EXL3_ERR_INVALID_ARG;
+        if (t.n_out % 128) return EXL3_ERR_UNSUPPORTED;
+        if (!aligned16(t.packed) || !aligned16(t.scale) || !aligned16(t.sv) || !aligned16(t.y))
+            return EXL3_ERR_MISALIGNED;
+        a.sib[i] = exl3::Sibling{t.packed, t.scale, t.sv, t.y, t.n_out, (int)(total / 128)};
+        total += t.n_out;
+    }
+    if (total > (1LL << 30)) return EXL3_ERR_UNSUPPORTED;
+    const int n_total = (int)total;
+    if (!workspace || ws_bytes < exl3_workspace_bytes(m, k_in, n_total, bits)) return EXL3_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
+    int st = check_arch();
+    if (st != EXL3_OK) return st;
+    a.x = x;
+    a.su = su;
+    a.y_fp32 = y_fp32 ? 1 : 0;
+    a.m = m;
+    a.k_in = k_in;
+    a.bits = bits;
+    a.n_out = n_total;
+    a.nsib = n_mats;
+    a.ws = static_cast<unsigned char*>(workspace);
+    a.pdl = 1;
+    cudaError_t e = m == 1 ? exl3::launch_gemv_m1(a, static_cast<cudaStream_t>(stream))
+                           : exl3::launch_gemm_tc(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------ no-allocation GEMV ---
 //
 // exl3_gemv_noalloc: the single-row product without a caller workspace, for
@@ -231,19 +281,7 @@ extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, cons
     // arrival counters must start at zero
     cudaError_t e = cudaMemsetAsync(ws, 0, exl3::ws_part_off(n_out), s);
     if (e != cudaSuccess) return cuda_fail(e);
-    exl3::GemmArgs a;
-    a.x = x;
-    a.packed = packed;
-    a.scale = scale;
-    a.su = su;
-    a.sv = sv;
-    a.y = y;
-    a.y_fp32 = y_fp32 ? 1 : 0;
-    a.m = 1;
-    a.k_in = k_in;
-    a.n_out = n_out;
-    a.bits = bits;
-    a.ws = static_cast<unsigned char*>(ws);
+    exl3::GemmArgs a = single_args(1, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws);
     a.pdl = 0;                       // follows a memset: ordinary stream order
     e = exl3::launch_gemv_m1(a, s);
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);

@@ -11,19 +11,56 @@ cudaError_t launch_decode_tiles(const uint32_t* packed, int k_in, int n_out, int
 cudaError_t launch_hadamard128(const uint16_t* in, uint16_t* out, const uint16_t* signs, int rows, int n, int mode,
                                cudaStream_t stream);
 
+// One product of a sibling group: the matrices that share the input x (and
+// its sign vector su), e.g. the gate and up projections of an MLP, or q, k
+// and v.  Output blocks of the group are numbered consecutively: sibling i
+// owns blocks [g0, g0 + n_out / 128).
+constexpr int kMaxSiblings = 8;
+struct Sibling {
+    const uint32_t* packed;   // trellis words (k_in x n_out)
+    const uint16_t* scale;    // n_out fp16
+    const uint16_t* sv;       // n_out fp16 +-1
+    void* y;                  // m x n_out, fp16 or fp32
+    int n_out;
+    int g0;                   // first output block of this sibling
+};
+
 // Problem description shared by the product kernels.
 struct GemmArgs {
     const uint16_t* x;        // m x k_in fp16
-    const uint32_t* packed;   // trellis words
-    const uint16_t* scale;    // n_out fp16
     const uint16_t* su;       // k_in fp16 +-1
-    const uint16_t* sv;       // n_out fp16 +-1
-    void* y;                  // m x n_out, fp16 or fp32
     int y_fp32;
-    int m, k_in, n_out, bits;
+    int m, k_in, bits;
+    int n_out;                // total output width of the group (sum over siblings)
+    int nsib;                 // 1 .. kMaxSiblings
+    Sibling sib[kMaxSiblings];
     unsigned char* ws;        // workspace base
     int pdl;                  // launch with programmatic dependent launch (overlap the previous kernel's tail)
 };
+
+#ifdef __CUDACC__
+// The sibling holding group output block g, and g's block index inside it.
+// Unrolled over the fixed-size table (no dynamically indexed parameters).
+struct SibView {
+    const uint32_t* packed;
+    const uint16_t* scale;
+    const uint16_t* sv;
+    void* y;
+    int n_out;
+    int gl;
+};
+__device__ __forceinline__ SibView sibling_of(const GemmArgs& a, int g)
+{
+    SibView v{a.sib[0].packed, a.sib[0].scale, a.sib[0].sv, a.sib[0].y, a.sib[0].n_out, g};
+#pragma unroll
+    for (int t = 1; t < kMaxSiblings; ++t) {
+        if (t < a.nsib && g >= a.sib[t].g0) {
+            v = SibView{a.sib[t].packed, a.sib[t].scale, a.sib[t].sv, a.sib[t].y, a.sib[t].n_out, g - a.sib[t].g0};
+        }
+    }
+    return v;
+}
+#endif
 
 // Single-row product on CUDA cores (gemv_m1.cu).
 size_t m1_workspace_bytes(int k_in, int n_out, int bits);

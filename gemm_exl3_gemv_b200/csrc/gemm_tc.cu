@@ -225,9 +225,10 @@ __device__ __forceinline__ void reduce_segments(const float* part, int g, int p_
 // channels 4*lane .. +3) times scale, output rotation, signs, store.
 __device__ __forceinline__ void finish_row_regs(const GemmArgs& a, int g, int mm, const float (&z)[4], int lane)
 {
-    const int n0 = 128 * g + 4 * lane;
-    const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
-    const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
+    const SibView sib = sibling_of(a, g);                 // the matrix holding block g
+    const int n0 = 128 * sib.gl + 4 * lane;
+    const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
+    const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
     const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
     const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
     const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
@@ -238,12 +239,12 @@ __device__ __forceinline__ void finish_row_regs(const GemmArgs& a, int g, int mm
     vv[1] *= kInvSqrt128 * sg0.y;
     vv[2] *= kInvSqrt128 * sg1.x;
     vv[3] *= kInvSqrt128 * sg1.y;
-    const size_t yo = (size_t)mm * a.n_out + n0;
+    const size_t yo = (size_t)mm * sib.n_out + n0;
     if (a.y_fp32) {
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(sib.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
     } else {
         __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
-        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + yo) = *reinterpret_cast<uint2*>(hh);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(sib.y) + yo) = *reinterpret_cast<uint2*>(hh);
     }
 }
 
@@ -274,7 +275,6 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int S = prm.S, C = prm.C;
     const int p = blockIdx.x;
-    const int tiles_n = a.n_out / 16;
     // this CTA's units [b0, b1) in block-major order
     long long b0, b1;
     if (S > 0) {
@@ -360,8 +360,10 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             const int c0 = (int)(u0 - (long long)g * C);
             const long long u1 = ((long long)(g + 1) * C < b1) ? (long long)(g + 1) * C : b1;
             const int nseg = (int)(u1 - u0);
+            const SibView sib = sibling_of(a, g);                      // the matrix holding block g
+            const int tiles_n = sib.n_out / 16;
             const uint32_t* src =
-                a.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
+                sib.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)sib.gl) * TW + (size_t)lane * QW;
             const size_t unit_step = (size_t)8 * tiles_n * TW;    // words between consecutive units
             bool ok = true;                                      // warp-uniform
             // decode the segment's unit k (the CTA's kk-th) from `wds` into A

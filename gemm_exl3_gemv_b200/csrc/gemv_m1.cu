@@ -141,10 +141,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     const int p = blockIdx.x;
     const int T = pl.T;
     const long long b0 = (long long)p * pl.U / pl.P, b1 = (long long)(p + 1) * pl.U / pl.P;
-    const int tiles_n = a.n_out / 16;
     const int q = lane & 3;
     const int src_prev = (lane & ~3) | ((q + 3) & 3);
-    const size_t row_step = (size_t)kM1Warps * tiles_n * TW;          // words between a warp's rows
     float* part = reinterpret_cast<float*>(a.ws + ws_part_off(a.n_out));
     uint32_t* counters = reinterpret_cast<uint32_t*>(a.ws + ws_counter_off());
     grid_dep_launch();                     // the next product may start loading its weights
@@ -159,8 +157,14 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         const int kb_lo = r0 >> 3, kb_hi = (r1 + 7) >> 3;             // 128-row input blocks touched
         const int nrow = r1 - r0;
         const int nw = nrow > warp ? (nrow - warp + kM1Warps - 1) / kM1Warps : 0;
-        const uint32_t* src =
-            a.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW;
+        size_t row_step;                                               // words between a warp's rows
+        const uint32_t* src;
+        {
+            const SibView sw = sibling_of(a, g);                       // the matrix holding block g
+            const int tiles_n = sw.n_out / 16;
+            row_step = (size_t)kM1Warps * tiles_n * TW;
+            src = sw.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)sw.gl) * TW + (size_t)lane * QW;
+        }
         uint32_t wa[QW], wb[QW];
         if (nw > 0) load_lane_words<BITS>(wa, src);                       // in flight during the rotation
         if (first_seg) grid_dep_wait();    // weights are never written; x, y, workspace only after this
@@ -272,10 +276,11 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
 
         // ---- epilogue (warp 0): scale, output rotation, signs, store ----
         if (warp == 0) {
-            const int n0 = 128 * g + 4 * lane;
+            const SibView sib = sibling_of(a, g);
+            const int n0 = 128 * sib.gl + 4 * lane;
             const float4 z4 = *reinterpret_cast<const float4*>(red + 4 * lane);
-            const uint2 sc = *reinterpret_cast<const uint2*>(a.scale + n0);
-            const uint2 sg = *reinterpret_cast<const uint2*>(a.sv + n0);
+            const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
+            const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
             const float2 sc0 = __half22float2(as_h2(sc.x)), sc1 = __half22float2(as_h2(sc.y));
             const float2 sg0 = __half22float2(as_h2(sg.x)), sg1 = __half22float2(as_h2(sg.y));
             float v[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
@@ -285,10 +290,10 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
             v[2] *= kInvSqrt128 * sg1.x;
             v[3] *= kInvSqrt128 * sg1.y;
             if (a.y_fp32) {
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.y) + n0) = make_float4(v[0], v[1], v[2], v[3]);
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(sib.y) + n0) = make_float4(v[0], v[1], v[2], v[3]);
             } else {
                 __half2 h[2] = {__floats2half2_rn(v[0], v[1]), __floats2half2_rn(v[2], v[3])};
-                *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(a.y) + n0) = *reinterpret_cast<uint2*>(h);
+                *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(sib.y) + n0) = *reinterpret_cast<uint2*>(h);
             }
         }
     }
@@ -302,11 +307,13 @@ M1Plan m1_plan(int k_in, int n_out, int bits)
     pl.T = k_in / 16;
     pl.U = (long long)G * pl.T;
     const long long slots = (long long)kSms * per_sm;   // one wave of resident CTAs
-    // With at most `slots` blocks, give every block the same whole number of
-    // CTAs, so that no range straddles two blocks (one segment per CTA: the
-    // per-segment costs -- input rotation, reduction, arrival -- are paid
-    // once); with more blocks, cut evenly across blocks.
+    // Give every block the same whole number of CTAs, so that no range
+    // straddles two blocks (one segment per CTA: the per-segment costs --
+    // input rotation, reduction, arrival -- are paid once), unless that
+    // leaves more than a tenth of the slots idle; then cut evenly across
+    // blocks (stream-K).
     long long P = G <= slots ? (long long)G * (slots / G) : slots;
+    if (10 * P < 9 * slots) P = slots;                  // whole-block split would idle >10 % of the slots
     if (P > pl.U / kM1Warps) P = pl.U / kM1Warps;       // at least one tile row per warp
     const long long rows_cap = 1024;                    // bounds the rotated input kept in shared memory
     if (P < (pl.U + rows_cap - 1) / rows_cap) P = (pl.U + rows_cap - 1) / rows_cap;

@@ -28,7 +28,7 @@ EXL3_ERR_TIMEOUT = 7
 # every entry point include/exl3.h declares
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",
            "exl3_workspace_status", "exl3_kernel_launches", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
-           "exl3_gemm_small_m", "exl3_gemv_noalloc")
+           "exl3_gemm_small_m", "exl3_gemm_siblings", "exl3_gemv_noalloc")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libexl3.so not built ({LIB_PATH}); run `python -m gemm_exl3_gemv_b200.build`")
@@ -56,6 +56,15 @@ lib.exl3_gemv.restype = _I
 lib.exl3_gemm_small_m.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]
 lib.exl3_gemm_small_m.restype = _I
 lib.exl3_gemv_noalloc.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P]
+
+
+class Matrix(ctypes.Structure):
+    """exl3_matrix_t: one member of a sibling group (device pointers)."""
+    _fields_ = [("packed", _P), ("scale", _P), ("sv", _P), ("y", _P), ("n_out", _I)]
+
+
+lib.exl3_gemm_siblings.argtypes = [_I, _P, _P, ctypes.POINTER(Matrix), _I, _I, _I, _I, _P, _Z, _P]
+lib.exl3_gemm_siblings.restype = _I
 lib.exl3_gemv_noalloc.restype = _I
 
 
@@ -146,3 +155,26 @@ def gemm(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, su: torch.T
                                    ws_bytes, _stream(stream))
         _check(st, "exl3_gemm_small_m")
     return out.reshape(-1) if squeeze else out
+
+
+def gemm_siblings(x: torch.Tensor, su: torch.Tensor, mats, bits: int, outs=None, fp32: bool = False,
+                  workspace: Optional[torch.Tensor] = None, stream=None):
+    """Products of one input with a group of matrices in one pass.  `mats` is a
+    list of (packed, scale, sv); returns the list of outputs (m, n_out_i)."""
+    squeeze = x.dim() == 1
+    x2 = x.reshape(1, -1) if squeeze else x
+    m, k_in = x2.shape
+    if outs is None:
+        outs = [torch.empty((m, sc.shape[0]), dtype=torch.float32 if fp32 else torch.float16, device=x.device)
+                for (_, sc, _) in mats]
+    n_total = sum(int(sc.shape[0]) for (_, sc, _) in mats)
+    if workspace is None:
+        workspace = alloc_workspace(m, k_in, n_total, bits, device=x.device)
+    arr = (Matrix * len(mats))()
+    for i, ((packed, scale, sv), y) in enumerate(zip(mats, outs)):
+        arr[i] = Matrix(packed.data_ptr(), scale.data_ptr(), sv.data_ptr(), y.data_ptr(), int(scale.shape[0]))
+    st = lib.exl3_gemm_siblings(m, _ptr(x2), _ptr(su), arr, len(mats), int(fp32), k_in, bits, _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "exl3_gemm_siblings")
+    return [o.reshape(-1) for o in outs] if squeeze else outs
+

@@ -159,6 +159,36 @@ EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
                       void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * exl3_gemm_siblings -- the product for a group of matrices that take the
+ * same input: y_i = sv_i .* H(scale_i .* (H(su .* x) W_i)) for i < n_mats,
+ * in one pass that rotates x once and spreads all the groups' output blocks
+ * over the GPU together.  This is the sibling fusion the exl3-rdna4-recipe
+ * page describes for verify batches ("a fused C++ MLP path", section "What we
+ * added on top of upstream"): gate and up of an MLP, or q, k and v of an
+ * attention block, whose inputs are the same activation rows.
+ *   x, su  : as exl3_gemm_small_m, shared by every matrix of the group.
+ *   mats   : HOST array of n_mats (1..8) exl3_matrix_t; each gives its packed
+ *            words, scale, sv and output y (m x n_out, row-major) and n_out
+ *            (a positive multiple of 128).  All matrices have k_in rows and
+ *            `bits` bits per weight.
+ *   workspace, ws_bytes : at least exl3_workspace_bytes(m, k_in, sum of n_out,
+ *            bits) bytes, zero-filled before first use.
+ * Results equal the separate products within rounding (the reduction split
+ * follows the group's total width); repeated calls are bitwise identical.
+ */
+typedef struct exl3_matrix {
+    const uint32_t *packed;
+    const uint16_t *scale;
+    const uint16_t *sv;
+    void *y;
+    int n_out;
+} exl3_matrix_t;
+
+EXL3_API int exl3_gemm_siblings(int m, const uint16_t *x, const uint16_t *su, const exl3_matrix_t *mats,
+                                int n_mats, int y_fp32, int k_in, int bits, void *workspace, size_t ws_bytes,
+                                void *stream);
+
+/*
  * exl3_gemv_noalloc -- exl3_gemv without a workspace argument.  The paper has
  * no counterpart of this entry point; it exists for callers that cannot
  * allocate device memory on the call path -- for example an inference engine

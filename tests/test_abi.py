@@ -101,3 +101,28 @@ def test_product_path_has_no_oracle_or_cpu_fallback():
             if f.endswith((".py", ".cu", ".cuh", ".h")) and f != "synth.py":
                 src = open(os.path.join(dirpath, f)).read()
                 assert "oracle" not in src.lower() or f == "__init__.py", f
+
+
+def test_siblings_validation(ex):
+    f = ex.lib.exl3_gemm_siblings
+    M = ex.Matrix
+
+    def mats(*n_outs, ptr=16):
+        arr = (M * max(1, len(n_outs)))()
+        for i, n in enumerate(n_outs):
+            arr[i] = M(ptr, ptr, ptr, ptr, n)
+        return arr
+
+    ws_ok = 1 << 26
+    call = lambda m, arr, n, k=256, bits=3, ws=256, wsb=ws_ok: f(m, P(16), P(16), arr, n, 0, k, bits, P(ws), wsb, None)
+    assert call(1, mats(256), 0) == ex.EXL3_ERR_INVALID_ARG                 # no matrices
+    assert call(1, mats(*([128] * 9)), 9) == ex.EXL3_ERR_UNSUPPORTED       # more than 8
+    assert call(1, mats(256, 200), 2) == ex.EXL3_ERR_UNSUPPORTED           # n_out not a multiple of 128
+    assert call(1, mats(256, 0), 2) == ex.EXL3_ERR_INVALID_ARG             # empty member
+    assert call(1, mats(256, 256, ptr=24), 2) == ex.EXL3_ERR_MISALIGNED    # member pointer misaligned
+    assert call(1, mats(256, 256), 2, k=200) == ex.EXL3_ERR_UNSUPPORTED    # k_in not a multiple of 128
+    assert call(33, mats(256), 1) == ex.EXL3_ERR_UNSUPPORTED               # too many rows
+    assert call(1, mats(256, 256), 2, wsb=64) == ex.EXL3_ERR_WORKSPACE     # sized for the group's total width
+    need = ex.workspace_bytes(32, 256, 512, 3)
+    assert call(32, mats(256, 256), 2, wsb=need - 1) == ex.EXL3_ERR_WORKSPACE
+    assert call(1, mats(256, 256), 2, ws=16) == ex.EXL3_ERR_MISALIGNED
