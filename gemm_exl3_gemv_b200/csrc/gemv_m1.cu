@@ -310,10 +310,10 @@ M1Plan m1_plan(int k_in, int n_out, int bits)
     // Give every block the same whole number of CTAs, so that no range
     // straddles two blocks (one segment per CTA: the per-segment costs --
     // input rotation, reduction, arrival -- are paid once), unless that
-    // leaves more than a tenth of the slots idle; then cut evenly across
-    // blocks (stream-K).
+    // leaves more than 15 % of the slots idle; then cut evenly across blocks
+    // (stream-K).
     long long P = G <= slots ? (long long)G * (slots / G) : slots;
-    if (10 * P < 9 * slots) P = slots;                  // whole-block split would idle >10 % of the slots
+    if (20 * P < 17 * slots) P = slots;                 // whole-block split would idle >15 % of the slots
     if (P > pl.U / kM1Warps) P = pl.U / kM1Warps;       // at least one tile row per warp
     const long long rows_cap = 1024;                    // bounds the rotated input kept in shared memory
     if (P < (pl.U + rows_cap - 1) / rows_cap) P = (pl.U + rows_cap - 1) / rows_cap;
