@@ -10,11 +10,16 @@
 namespace exl3 {
 
 // ------------------------------------------------------------ workspace ---
-// [0, 256)            status word (uint32 at 0): nonzero after a timed-out wait
+// [0, 256)            status word (uint32 at 0): nonzero after a timed-out wait;
+//                     word 1 (uint32 at 4): timeout injection for tests -- while
+//                     it is nonzero the verify kernel issues no copies of the
+//                     rotated input, so every wait for one runs out (zero in
+//                     normal use: the workspace is zero-filled)
 // [256, 256 + 4*G)    one arrival counter per 128-channel output block
 // [ws_part_off, ...)  split-K partial sums, fp32 [splits][m][n_out]
 constexpr size_t kWsHeader = 256;
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr size_t kWsInjectOff = 4;
 
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 __host__ __device__ inline size_t ws_counter_off() { return kWsHeader; }

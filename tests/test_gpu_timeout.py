@@ -1,0 +1,34 @@
+"""Failure detection without a GPU fault: the multi-row kernel's bounded waits.
+The test withholds the rotated input through the workspace's injection word
+(a flag that nothing sets then), so every wait for it runs out after its 2 s
+limit; the kernel winds down and the host reads EXL3_ERR_TIMEOUT from the
+workspace status word.  The context stays usable: a normal call afterwards on
+the same workspace is correct."""
+import numpy as np
+import pytest
+
+from gemm_exl3_gemv_b200 import synth
+from gpu_helpers import check_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("k,n", [(640, 256), (256, 65536)])     # cluster cut; stream-K cut
+def test_withheld_input_times_out_and_reports(oracle_mod, k, n):
+    import torch
+    from gemm_exl3_gemv_b200 import exl3 as ex
+    m, bits = 8, 3
+    spec = synth.MatrixSpec("to", k, n, bits, m, seed=71)
+    inp = synth.make_inputs(spec)
+    args = [to_dev(a) for a in (inp.x, inp.packed, inp.scale, inp.su, inp.sv)]
+    ws = ex.alloc_workspace(m, k, n, bits)
+    ws[4:8] = 1                                   # inject: withhold the rotated input
+    ex.gemm(*args, bits, fp32=True, workspace=ws)
+    assert ex.workspace_status(ws) == ex.EXL3_ERR_TIMEOUT
+    ws[4:8] = 0
+    y = ex.gemm(*args, bits, fp32=True, workspace=ws)
+    assert ex.workspace_status(ws) == ex.EXL3_OK
+    blocks = [0, n // 128 - 1]
+    ref = oracle_mod.gemm_sampled(inp.x, inp.packed, inp.scale, inp.su, inp.sv, k, n, bits, blocks)
+    yv = y.cpu().numpy().astype(np.float64)
+    check_close(np.concatenate([yv[:, 128 * b:128 * (b + 1)] for b in blocks], axis=1), ref, "after timeout")
