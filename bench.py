@@ -47,6 +47,8 @@ def parse():
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-budget", type=float, default=None,
+                    help="seconds of oracle work per step for --impl reference (default: about 90 s per run)")
     ap.add_argument("--only", default=None,
                     help="restrict the stack to one matrix kind (q,k,v,o,gate,up,down), e.g. for ncu captures")
     return ap.parse_args()
@@ -192,7 +194,7 @@ def run_reference(args, world, rank):
     os.environ.setdefault("OMP_NUM_THREADS", str(cores_used()))
     steps, warmup = args.steps, args.warmup
     # size each step so the whole run stays within a few minutes
-    per_step_budget = max(1.0, 90.0 / max(1, steps + warmup))
+    per_step_budget = args.ref_budget if args.ref_budget is not None else max(1.0, 90.0 / max(1, steps + warmup))
     vals, samples = [], None
     for i in range(warmup + steps):
         b, t, names = oracle_sample(per_step_budget, args.m)
