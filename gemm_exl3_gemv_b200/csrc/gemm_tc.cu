@@ -11,10 +11,10 @@
 //     laid out as the MMA's B operand (K-major, 128-byte swizzle), m padded to
 //     NT = 16 or 32 rows with zeros.
 //   * Unit = one 128-row block of K_in for one 128-channel output block: 8
-//     tile rows, 16384 weights.  Stream-K: the G x C units are cut into equal
-//     contiguous ranges, one per CTA, two CTAs per SM.  A range may cover the
-//     end of one block and the start of the next; each (CTA, block) piece is
-//     a segment.
+//     tile rows, 16384 weights.  Two ways to cut the units over the CTAs (two
+//     per SM), chosen per shape by a small cost model (see TcParams):
+//     clusters of S CTAs per output block that add their partial sums through
+//     distributed shared memory, or a stream-K cut with workspace partials.
 //   * Eight decoder warps.  Warp w decodes tile row w of every unit: lane l
 //     takes quarter l%4 of tile l/4 (64 consecutive weights) from its words,
 //     loaded straight from HBM into registers one unit ahead (coalesced: the
@@ -23,19 +23,22 @@
 //     stored into the warp's own A stage (128 channels x 16 k, MN-major,
 //     128-byte swizzle).  Lane 0 of the warp then issues the MMA itself --
 //     tcgen05.mma kind::f16, M = 128 channels, N = NT rows, K = 16 -- into the
-//     warp's own tensor-memory accumulator, and commits it to the stage's
-//     barrier.  No dedicated issuer warps and no polling: a warp waits only
-//     for its own stage (two units back) and for the unit's xt chunk.
-//   * A ninth warp streams the xt chunks (1-D bulk copies + mbarrier) into a
-//     two-stage ring shared by the eight decoders.
-//   * End of a segment: every warp reads its lane quarter of all eight
-//     accumulators (tcgen05.ld) and adds them in a fixed order.  A block
-//     split over several CTAs: each writes its partial sums to the workspace
-//     and the last to arrive (atomic counter, no waiting) adds them in CTA
-//     order -- fixed, so results are bitwise repeatable -- then scales,
-//     rotates and writes y.
+//     warp's own tensor-memory accumulator (so the accumulation order is
+//     fixed), and commits it to the stage's barrier.  A warp waits only for
+//     its own stage (two units back) and for the unit's xt.
+//   * A ninth warp streams each unit's xt (1-D bulk copies + mbarrier) into a
+//     four-stage ring shared by the eight decoders.
+//   * End of a block's share: the CTA reads all eight accumulators
+//     (tcgen05.ld) and adds them in a fixed order; the partial sums of a block
+//     split over several CTAs meet in rank / CTA order -- fixed, so results
+//     are bitwise repeatable -- then the finishing warps scale, rotate and
+//     write y.
+//   * Launched with programmatic dependent launch: set-up and the first word
+//     loads overlap the previous kernel; xt, y and the workspace are touched
+//     only after griddepcontrol.wait.
 //   * Every mbarrier wait is bounded (2 s); on expiry the CTA records a
-//     timeout in the workspace status word and winds down.
+//     timeout in the workspace status word and winds down through the same
+//     barriers (tested by withholding xt: see the workspace injection word).
 #include <atomic>
 #include <mutex>
 #include <utility>
