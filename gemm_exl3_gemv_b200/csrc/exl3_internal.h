@@ -1,6 +1,7 @@
 // exl3_internal.h -- launchers shared between the libexl3 translation units.
 #pragma once
 #include <cstddef>
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -61,6 +62,23 @@ __device__ __forceinline__ SibView sibling_of(const GemmArgs& a, int g)
     return v;
 }
 #endif
+
+// Kernel attributes (shared-memory limit, cluster size) are per device: a
+// process that drives several GPUs sets them once on each.  `done` is a
+// per-kernel table indexed by device; returns the first error.
+constexpr int kMaxDevices = 64;
+template <typename F>
+cudaError_t once_per_device(std::atomic<int> (&done)[kMaxDevices], F&& setup)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = setup();                                     // idempotent: a race only repeats it
+    if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+    return e;
+}
 
 // Single-row product on CUDA cores (gemv_m1.cu).
 size_t m1_workspace_bytes(int k_in, int n_out, int bits);

@@ -666,18 +666,18 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     if (e != cudaSuccess) return e;
 
     auto kern = gemm_tc_kernel<BITS, NT>;
-    static std::once_flag once;
-    static cudaError_t setup = cudaSuccess;
-    std::call_once(once, [&] {
-        setup = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
-        if (setup == cudaSuccess) setup = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-        if (setup == cudaSuccess)
-            setup = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         TcLayout<32>::total);
-        if (setup == cudaSuccess)
-            setup = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    static std::atomic<int> configured[kMaxDevices];
+    e = once_per_device(configured, [&] {
+        cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
+        if (r == cudaSuccess) r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     TcLayout<32>::total);
+        if (r == cudaSuccess)
+            r = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        return r;
     });
-    if (setup != cudaSuccess) return setup;
+    if (e != cudaSuccess) return e;
 
     // plan decided once per shape (host-side occupancy queries), then cached
     static std::mutex mu;

@@ -347,14 +347,12 @@ cudaError_t launch_m1_t(const GemmArgs& a, cudaStream_t stream)
     const M1Plan pl = m1_plan(a.k_in, a.n_out, a.bits);
     const size_t smem = m1_smem_bytes(pl);
     auto kern = gemv_m1_kernel<BITS, kAltEvery<BITS>>;
-    static std::atomic<int> configured{0};
-    if ((int)smem > configured.load()) {
-        const int lim = 200 * 1024;
-        if ((int)smem > lim) return cudaErrorInvalidValue;
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, lim);
-        if (e != cudaSuccess) return e;
-        configured.store(lim);
-    }
+    static std::atomic<int> configured[kMaxDevices];
+    if ((int)smem > 200 * 1024) return cudaErrorInvalidValue;
+    cudaError_t ce = once_per_device(configured, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    });
+    if (ce != cudaSuccess) return ce;
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
