@@ -11,7 +11,8 @@
  *   The pages name the format ("~3.2 bits/weight in the EXL3 trellis format",
  *   orcasaq2-rocm README, opening paragraph; "EXL3, 3.0 bpw ... SC_3.00bpw_H4",
  *   exl3-rdna4-recipe, opening paragraph) but never define it.  The definition
- *   written out below is the task specification's: 16x16 tiles, each a
+ *   written out below is the format specification this library follows:
+ *   16x16 tiles, each a
  *   tail-biting bitstream of 256*K bits; weight i of a tile is decoded from the
  *   16-bit window ending at bit (i+1)*K with the 3INST map
  *       x = state*89226354 + 64248484 (mod 2^32),
