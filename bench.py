@@ -61,7 +61,8 @@ def dist_env():
     return world, rank, local
 
 
-KERNEL_SOURCES = ["gemm_exl3_gemv_b200/csrc/gemm_tc.cu", "gemm_exl3_gemv_b200/csrc/exl3_decode.cuh",
+KERNEL_SOURCES = ["gemm_exl3_gemv_b200/csrc/gemm_tc.cu", "gemm_exl3_gemv_b200/csrc/exl3_aop.cuh",
+                  "gemm_exl3_gemv_b200/csrc/exl3_decode.cuh",
                   "gemm_exl3_gemv_b200/csrc/exl3_common.cuh", "gemm_exl3_gemv_b200/csrc/exl3_tc.cuh"]
 
 

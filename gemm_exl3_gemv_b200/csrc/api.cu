@@ -176,6 +176,33 @@ int exl3_gemm_small_m(int m, const uint16_t* x, const uint32_t* packed, const ui
 
 }  // extern "C"
 
+// ----------------------------------------------------------------- large m ---
+
+extern "C" size_t exl3_large_m_workspace_bytes(int m, int k_in, int n_out, int bits)
+{
+    if (m <= 0 || m > (1 << 20) || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
+    return exl3::large_workspace_bytes(m, k_in, n_out);
+}
+
+extern "C" int exl3_gemm_large_m(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale,
+                                 const uint16_t* su, const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out,
+                                 int bits, void* workspace, size_t ws_bytes, void* stream)
+{
+    if (!x || !packed || !scale || !su || !sv || !y) return EXL3_ERR_INVALID_ARG;
+    if (m <= 0 || k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
+    if (m > (1 << 20) || !bits_ok(bits) || k_in % 128 || n_out % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(su) || !aligned16(sv) ||
+        !aligned16(y))
+        return EXL3_ERR_MISALIGNED;
+    if (!workspace || ws_bytes < exl3_large_m_workspace_bytes(m, k_in, n_out, bits)) return EXL3_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
+    int st = check_arch();
+    if (st != EXL3_OK) return st;
+    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, workspace);
+    cudaError_t e = exl3::launch_gemm_large(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
 // ------------------------------------------------------------- siblings ---
 
 extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, const exl3_matrix_t* mats,

@@ -91,4 +91,12 @@ int tc_ctas(int m, int k_in, int n_out, int bits);
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
 
+// Many-row path (gemm_large.cu): decode once into the tensor-core operand
+// image, then a tcgen05 GEMM.  Rows per tile (256, 128 or 64: the largest that
+// still gives kLargeMinCtas tiles), workspace size, launcher (three launches).
+constexpr int kLargeMinCtas = 148;
+int large_tile_rows(int m, int n_out);
+size_t large_workspace_bytes(int m, int k_in, int n_out);
+cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream);
+
 }  // namespace exl3

@@ -1,0 +1,392 @@
+// gemm_large.cu -- the product for many input rows (prompt prefill): decode the
+// whole matrix once into the tensor-core operand layout, then a tcgen05 GEMM.
+//
+// What is computed (the prompt-processing side of the decode speeds on the
+// orcasaq2-rocm README -- "Prefill: 1100-1800 tok/s at 8-32k", paragraph below
+// its speed table -- and of the exl3-rdna4-recipe page, "What you get"):
+//     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: m x K_in, y: m x N_out
+// At large m each decoded weight feeds 2m flops, so the decode is paid once per
+// call and the contraction runs as a dense tensor-core GEMM:
+//   1. decode_aimage_kernel: every warp decodes one tile row of one 128-channel
+//      output block (as the verify kernel's decoders do) and writes it as the
+//      4 KB MN-major, 128-byte-swizzled A operand image the MMA reads, into the
+//      workspace: image (g, 64-row chunk c) = 16 KB = 4 tile rows, contiguous.
+//   2. xt_tiled_prepass_kernel: xt = H(su .* x) in fp16, laid out as the B
+//      operand (K-major, 128-byte swizzle) per tile of NB input rows:
+//      xt (j, c) = NB rows x 64 k = NB * 128 contiguous bytes, rows past m zero.
+//   3. gemm_large_kernel<NB>: CTA (g, j) computes output channels of block g for
+//      rows of tile j.  Warp 0 streams A and B chunks with 1-D bulk copies
+//      (cp.async.bulk + mbarrier) into a 3-stage ring; one thread of warp 1
+//      issues tcgen05.mma kind::f16 (M = 128 channels, N = NB rows, K = 16;
+//      four per 64-row chunk) into one tensor-memory accumulator; then the four
+//      warps drain it 16 rows at a time (tcgen05.ld), scale, rotate, store y.
+//   No split-K: each output element is one accumulator's fixed-order sum, so
+//   results are bitwise repeatable.  Every wait is bounded (2 s).
+#include <atomic>
+
+#include "exl3_aop.cuh"
+#include "exl3_common.cuh"
+#include "exl3_decode.cuh"
+#include "exl3_internal.h"
+#include "exl3_tc.cuh"
+
+namespace exl3 {
+
+namespace {
+
+constexpr int kLgThreads = 128;
+constexpr int kLgStages = 3;
+constexpr int kAChunk = 16384;                 // A image of one 64-row chunk of one output block
+constexpr uint64_t kLgWaitNs = 2000000000ull;
+
+// ------------------------------------------------------------- 1. decode ---
+template <int BITS>
+__global__ void __launch_bounds__(256) decode_aimage_kernel(const uint32_t* __restrict__ packed, int k_in, int n_out,
+                                                            uint8_t* __restrict__ image, uint32_t two16)
+{
+    constexpr int TW = 8 * BITS, QW = 2 * BITS;
+    grid_dep_wait();                                  // the image is read by the previous call's GEMM
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int T = k_in / 16, tiles_n = n_out / 16;
+    const long long item = (long long)blockIdx.x * 8 + warp;   // (block g, tile row tr)
+    if (item >= (long long)(n_out / 128) * T) return;
+    const int g = (int)(item / T), tr = (int)(item % T);
+    uint32_t w[QW];
+    load_lane_words<BITS>(w, packed + ((size_t)tr * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW);
+    const int q = lane & 3;
+    uint32_t buf[QW + 1];
+    buf[0] = __shfl_sync(0xffffffffu, w[QW - 1], (lane & ~3) | ((q + 3) & 3));
+#pragma unroll
+    for (int t = 0; t < QW; ++t) buf[t + 1] = w[t];
+    uint32_t soff[2][2];
+    lane_soff(lane, soff);
+    uint8_t* dst = image + ((size_t)g * T + tr) * 4096;
+    decode_quarter_to_a<BITS>(buf, soff, two16, [&](uint32_t off, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
+        *reinterpret_cast<uint4*>(dst + off) = make_uint4(w0, w1, w2, w3);
+    });
+    grid_dep_launch();
+}
+
+// ---------------------------------------------------------- 2. pre-pass ---
+// Same rotation and in-chunk layout as the verify kernel's pre-pass (within
+// each 16-row group, k = 4q + r sits at position 8(r >> 1) + 4(r & 1) + q, to
+// match the A image), tiled by NB input rows.
+__global__ void __launch_bounds__(256) xt_tiled_prepass_kernel(const __half* __restrict__ x,
+                                                               const __half* __restrict__ su, int m_rows,
+                                                               int m_pad, int k_in, int nb, uint8_t* __restrict__ xt)
+{
+    grid_dep_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = k_in / 128;
+    const long long item = (long long)blockIdx.x * 8 + warp;
+    if (item >= (long long)m_pad * nblk) return;
+    const int m = (int)(item / nblk), b = (int)(item % nblk);
+    float v[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int k = 128 * b + ((lane & 3) | (e << 2) | ((lane >> 2) << 4));
+        v[e] = (m < m_rows) ? __half2float(x[(size_t)m * k_in + k]) * __half2float(su[k]) : 0.f;
+    }
+    fwht128_warp(v);
+    const int tr = 8 * b + (lane >> 2);
+    const int pk0 = 16 * tr + 8 * ((lane >> 1) & 1) + 4 * (lane & 1);
+    const int kchunk = pk0 >> 6, o = pk0 & 63, c16 = o >> 3, pos = o & 7;
+    const int j = m / nb, mr = m % nb;
+    uint8_t* dst = xt + ((size_t)j * (k_in / 64) + kchunk) * nb * 128 + (mr >> 3) * 1024 + (mr & 7) * 128 +
+                   ((c16 ^ (mr & 7)) << 4) + pos * 2;
+    __half2 h2[2] = {__floats2half2_rn(v[0] * kInvSqrt128, v[1] * kInvSqrt128),
+                     __floats2half2_rn(v[2] * kInvSqrt128, v[3] * kInvSqrt128)};
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<uint2*>(h2);
+    grid_dep_launch();
+}
+
+// --------------------------------------------------------------- 3. GEMM ---
+template <int NB>
+struct LgLayout {
+    static constexpr int BCHUNK = NB * 128;                 // B bytes per 64-row chunk
+    static constexpr int STAGE = kAChunk + BCHUNK;
+    static constexpr int off_stage = 0;
+    static constexpr int off_z = off_stage + kLgStages * STAGE;   // z [16][128] fp32
+    static constexpr int off_bar = off_z + 16 * 128 * 4;
+    static constexpr int nbar = 2 * kLgStages + 1;          // full[], empty[], done
+    static constexpr int off_misc = off_bar + nbar * 8;
+    static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
+    static_assert(STAGE % 1024 == 0 && off_z % 1024 == 0, "layout");
+    static_assert(total <= 227 * 1024, "shared memory");
+    // NB <= 256 columns of tensor memory; with at most two CTAs of this size
+    // per SM (shared memory), allocations never wait
+    static_assert(NB == 64 || NB == 128 || NB == 256, "tensor memory columns");
+};
+
+struct LgParams {
+    const uint8_t* image;     // decoded A images
+    const uint8_t* xt;        // B images
+    const uint16_t* scale;
+    const uint16_t* sv;
+    void* y;
+    uint32_t* status;
+    int y_fp32, m, k_in, n_out;
+};
+
+__device__ __forceinline__ bool lg_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    while (true) {
+        for (int i = 0; i < 16; ++i)
+            if (mbar_try_wait_sleep(bar, parity, 1000)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kLgWaitNs) {
+            atomicExch((int*)abort_flag, 1);
+            return false;
+        }
+    }
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
+{
+    using L = LgLayout<NB>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::off_bar);
+    uint64_t* empty = full + kLgStages;
+    uint64_t* done = empty + kLgStages;
+    int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
+    volatile int* abort_flag = misc + 1;
+    float* zsm = reinterpret_cast<float*>(smem + L::off_z);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = prm.n_out / 128;
+    const int g = blockIdx.x % G, j = blockIdx.x / G;
+    const int C64 = prm.k_in / 64;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kLgStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        mbar_init(done, 1);
+        misc[1] = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), NB);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = (uint32_t)misc[0];
+    grid_dep_wait();                                   // A and B images are the pre-passes' output
+
+    if (warp == 0 && lane == 0) {
+        // ---- producer: A and B chunks of this tile into the stage ring ----
+        const uint8_t* a_src = prm.image + (size_t)g * C64 * kAChunk;
+        const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
+        int issued = 0;
+        for (int c = 0; c < C64; ++c) {
+            const int s = c % kLgStages;
+            if (c >= kLgStages && !lg_wait(&empty[s], (uint32_t)(c / kLgStages - 1) & 1u, abort_flag)) break;
+            mbar_arrive_expect_tx(&full[s], L::STAGE);
+            uint8_t* st = smem + L::off_stage + s * L::STAGE;
+            bulk_g2s(st, a_src + (size_t)c * kAChunk, kAChunk, &full[s]);
+            bulk_g2s(st + kAChunk, b_src + (size_t)c * L::BCHUNK, L::BCHUNK, &full[s]);
+            issued = c + 1;
+        }
+        // on abort, let every issued copy land before the CTA can exit
+        if (*abort_flag)
+            for (int v = issued > kLgStages ? issued - kLgStages : 0; v < issued; ++v)
+                (void)mbar_wait_bounded(&full[v % kLgStages], (uint32_t)(v / kLgStages) & 1u, 100000000ull);
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issuer: four K = 16 steps per chunk into the accumulator ----
+        constexpr uint32_t idesc = idesc_f16_amn(128, NB);
+        bool ok = true;
+        for (int c = 0; c < C64 && ok; ++c) {
+            const int s = c % kLgStages;
+            if (!lg_wait(&full[s], (uint32_t)(c / kLgStages) & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t st = smem_u32(smem + L::off_stage + s * L::STAGE);
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+                mma_f16_ss(tmem, sdesc_sw128(st + t * 4096, 1024, 2048), sdesc_sw128(st + kAChunk + t * 32, 16, 1024),
+                           idesc, (c > 0 || t > 0) ? 1u : 0u);
+            mma_commit(&empty[s]);
+        }
+        if (ok) mma_commit(done);
+        else mbar_arrive(done);
+    }
+    __syncwarp();
+
+    // ---- epilogue: 16 rows at a time, accumulator -> z -> y ----
+    int okd = 1;
+    if (lane == 0) okd = lg_wait(done, 0u, abort_flag) ? 1 : 0;
+    okd = __shfl_sync(0xffffffffu, okd, 0);
+    tc_fence_after();
+    const int ch = chan_of_row(32 * warp + lane);
+    for (int t0 = 0; t0 < NB; t0 += 16) {
+        if (j * NB + t0 >= prm.m) break;                  // uniform: rows past m are padding
+        uint32_t t16[16];
+        if (okd) {
+            tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)t0, t16);
+            tmem_ld_wait();
+        } else {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) t16[t] = 0u;
+        }
+#pragma unroll
+        for (int t = 0; t < 16; ++t) zsm[t * 128 + ch] = __uint_as_float(t16[t]);
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int mm = j * NB + t0 + 4 * warp + i;
+            if (mm >= prm.m) break;
+            const int n0 = 128 * g + 4 * lane;
+            const float4 z4 = *reinterpret_cast<const float4*>(zsm + (4 * warp + i) * 128 + 4 * lane);
+            const uint2 sc = *reinterpret_cast<const uint2*>(prm.scale + n0);
+            const uint2 sg = *reinterpret_cast<const uint2*>(prm.sv + n0);
+            const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+            const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+            const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+            const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+            float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
+            fwht128_warp(vv);
+            vv[0] *= kInvSqrt128 * sg0.x;
+            vv[1] *= kInvSqrt128 * sg0.y;
+            vv[2] *= kInvSqrt128 * sg1.x;
+            vv[3] *= kInvSqrt128 * sg1.y;
+            const size_t yo = (size_t)mm * prm.n_out + n0;
+            if (prm.y_fp32) {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
+            } else {
+                __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
+                *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(prm.y) + yo) = *reinterpret_cast<uint2*>(hh);
+            }
+        }
+        __syncthreads();
+    }
+    grid_dep_launch();
+
+    // ---- teardown ----
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, NB);
+    }
+    if (threadIdx.x == 0 && misc[1]) atomicOr(prm.status, kStatusTimeout);
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ host ---
+
+int large_tile_rows(int m, int n_out)
+{
+    const long long G = n_out / 128;
+    for (int nb : {256, 128}) {
+        if (G * ((m + nb - 1) / nb) >= kLargeMinCtas) return nb;
+    }
+    return 64;
+}
+
+size_t large_workspace_bytes(int m, int k_in, int n_out)
+{
+    const int nb = large_tile_rows(m, n_out);
+    const size_t m_pad = (size_t)((m + nb - 1) / nb) * nb;
+    return kWsHeader + (size_t)k_in * n_out * 2 + m_pad * k_in * 2;
+}
+
+namespace {
+
+template <int NB>
+cudaError_t launch_gemm_large_nb(const LgParams& prm, cudaStream_t stream, int pdl)
+{
+    using L = LgLayout<NB>;
+    auto kern = gemm_large_kernel<NB>;
+    static std::atomic<int> configured[kMaxDevices];
+    cudaError_t e = once_per_device(configured, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
+    });
+    if (e != cudaSuccess) return e;
+    const int G = prm.n_out / 128, J = (prm.m + NB - 1) / NB;
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)(G * J), 1, 1);
+    cfg.blockDim = dim3(kLgThreads, 1, 1);
+    cfg.dynamicSmemBytes = L::total;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
+template <int BITS>
+cudaError_t launch_decode_image(const uint32_t* packed, int k_in, int n_out, uint8_t* image, cudaStream_t stream,
+                                int pdl)
+{
+    const long long items = (long long)(n_out / 128) * (k_in / 16);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3((unsigned)((items + 7) / 8), 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, decode_aimage_kernel<BITS>, packed, k_in, n_out, image, 0x10000u);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
+{
+    const Sibling& sb = a.sib[0];
+    const int nb = large_tile_rows(a.m, a.n_out);
+    const int m_pad = (a.m + nb - 1) / nb * nb;
+    uint8_t* image = a.ws + kWsHeader;
+    uint8_t* xt = image + (size_t)a.k_in * a.n_out * 2;
+
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (a.bits) {
+        case 2: e = launch_decode_image<2>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
+        case 3: e = launch_decode_image<3>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
+        case 4: e = launch_decode_image<4>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
+    }
+    if (e != cudaSuccess) return e;
+    {
+        const long long items = (long long)m_pad * (a.k_in / 128);
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3((unsigned)((items + 7) / 8), 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = a.pdl ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, xt_tiled_prepass_kernel, reinterpret_cast<const __half*>(a.x),
+                               reinterpret_cast<const __half*>(a.su), a.m, m_pad, a.k_in, nb, xt);
+        if (e != cudaSuccess) return e;
+    }
+    LgParams prm;
+    prm.image = image;
+    prm.xt = xt;
+    prm.scale = sb.scale;
+    prm.sv = sb.sv;
+    prm.y = sb.y;
+    prm.status = reinterpret_cast<uint32_t*>(a.ws);
+    prm.y_fp32 = a.y_fp32;
+    prm.m = a.m;
+    prm.k_in = a.k_in;
+    prm.n_out = a.n_out;
+    switch (nb) {
+        case 256: e = launch_gemm_large_nb<256>(prm, stream, a.pdl); break;
+        case 128: e = launch_gemm_large_nb<128>(prm, stream, a.pdl); break;
+        default: e = launch_gemm_large_nb<64>(prm, stream, a.pdl); break;
+    }
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+}
+
+}  // namespace exl3

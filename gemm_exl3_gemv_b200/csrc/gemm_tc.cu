@@ -45,6 +45,7 @@
 
 #include <cooperative_groups.h>
 
+#include "exl3_aop.cuh"
 #include "exl3_common.cuh"
 #include "exl3_decode.cuh"
 #include "exl3_internal.h"
@@ -128,52 +129,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
             return false;
         }
     }
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d)
-{
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
-// Row v of an accumulator (row v of A) holds output channel chan_of_row(v):
-// tile j's 16 channels fill 16-byte chunks 4*(j&1) + 2*((j>>1)&1) + e of MN
-// atom j/4 (e = channel/8), so that the 8 lanes of a store phase hit 8
-// different banks.
-__host__ __device__ constexpr int chunk_of_tile(int j4, int e) { return 4 * (j4 & 1) + 2 * ((j4 >> 1) & 1) + e; }
-__device__ __forceinline__ int chan_of_row(int v)
-{
-    const int atom = v >> 6, chunk = (v >> 3) & 7, pos = v & 7;
-    const int j4 = 2 * ((chunk >> 1) & 1) + ((chunk >> 2) & 1);
-    return 16 * (4 * atom + j4) + 8 * (chunk & 1) + pos;
-}
-
-// Decode the 64 weights of quarter q of tile j (4 input rows x 16 channels)
-// into fp16 (the two halves of each 3INST word added and rounded once, RNE:
-// the exact decoded weight) and store them into the A stage at `ast`, two
-// 16-byte chunks per row.  soff[rb][e]: per-lane byte offset of the chunk
-// holding channels 8e..8e+7 of a row with (row & 1) == rb; row >> 1 selects
-// the 8-row K group (+2048 bytes).
-template <int BITS, int NW>
-__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], uint32_t ast,
-                                                    const uint32_t (&soff)[2][2], uint32_t two16)
-{
-    auto body = [&](auto R, auto E) {
-        constexpr int r = decltype(R)::value, e = decltype(E)::value;
-        // channels 8e + 2c, 8e + 2c + 1 of row r -> one fp16 pair
-        auto pair = [&](auto Cc) -> uint32_t {
-            constexpr int c = decltype(Cc)::value;
-            constexpr int ia = 16 * r + 8 * e + 2 * c, ib = ia + 1;
-            const uint32_t ma = inst3(window_auto<BITS, ia, (ia + 1) * BITS + 16>(buf, two16));
-            const uint32_t mb = inst3(window_auto<BITS, ib, (ib + 1) * BITS + 16>(buf, two16));
-            return weight_pair_h(ma, mb);
-        };
-        sts128(ast + soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
-               pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
-               pair(std::integral_constant<int, 3>{}));
-    };
-    [&]<int... RE>(std::integer_sequence<int, RE...>) {
-        (body(std::integral_constant<int, RE / 2>{}, std::integral_constant<int, RE % 2>{}), ...);
-    }(std::make_integer_sequence<int, 8>{});
 }
 
 // zsm[0 .. m*128) = sum of the partial slots (q + g) for q = p_first..p_last,
@@ -339,14 +294,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         const int q = lane & 3;
         const int src_prev = (lane & ~3) | ((q + 3) & 3);
         uint32_t soff[2][2];
-        {
-            const int j = lane >> 2, atom = j >> 2, j4 = j & 3;
-#pragma unroll
-            for (int rb = 0; rb < 2; ++rb)
-#pragma unroll
-                for (int e = 0; e < 2; ++e)
-                    soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
-        }
+        lane_soff(lane, soff);
         constexpr uint32_t idesc = idesc_f16_amn(128, NT);
         static_assert(kAStages == 2, "A stage index = unit counter & 1");
         static_assert((kBStages & (kBStages - 1)) == 0, "power of two");
@@ -388,7 +336,11 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 buf[0] = __shfl_sync(0xffffffffu, wds[QW - 1], src_prev);
 #pragma unroll
                 for (int t = 0; t < QW; ++t) buf[t + 1] = wds[t];
-                decode_quarter_to_a<BITS>(buf, s ? ast1 : ast0, soff, prm.two16);
+                const uint32_t ast = s ? ast1 : ast0;
+                decode_quarter_to_a<BITS>(buf, soff, prm.two16, [&](uint32_t off, uint32_t w0, uint32_t w1,
+                                                                    uint32_t w2, uint32_t w3) {
+                    sts128(ast + off, w0, w1, w2, w3);
+                });
                 fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
                 if (lane == 0) {

@@ -28,7 +28,8 @@ EXL3_ERR_TIMEOUT = 7
 # every entry point include/exl3.h declares
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",
            "exl3_workspace_status", "exl3_kernel_launches", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
-           "exl3_gemm_small_m", "exl3_gemm_siblings", "exl3_gemv_noalloc")
+           "exl3_gemm_small_m", "exl3_gemm_siblings", "exl3_large_m_workspace_bytes", "exl3_gemm_large_m",
+           "exl3_gemv_noalloc")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libexl3.so not built ({LIB_PATH}); run `python -m gemm_exl3_gemv_b200.build`")
@@ -65,6 +66,10 @@ class Matrix(ctypes.Structure):
 
 lib.exl3_gemm_siblings.argtypes = [_I, _P, _P, ctypes.POINTER(Matrix), _I, _I, _I, _I, _P, _Z, _P]
 lib.exl3_gemm_siblings.restype = _I
+lib.exl3_large_m_workspace_bytes.argtypes = [_I, _I, _I, _I]
+lib.exl3_large_m_workspace_bytes.restype = _Z
+lib.exl3_gemm_large_m.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]
+lib.exl3_gemm_large_m.restype = _I
 lib.exl3_gemv_noalloc.restype = _I
 
 
@@ -177,4 +182,24 @@ def gemm_siblings(x: torch.Tensor, su: torch.Tensor, mats, bits: int, outs=None,
                                 workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "exl3_gemm_siblings")
     return [o.reshape(-1) for o in outs] if squeeze else outs
+
+
+def gemm_large(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, su: torch.Tensor, sv: torch.Tensor,
+               bits: int, out: Optional[torch.Tensor] = None, fp32: bool = False,
+               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The product for many rows (x: m x k_in), decoding W once per call."""
+    m, k_in = x.shape
+    n_out = scale.shape[0]
+    if out is None:
+        out = torch.empty((m, n_out), dtype=torch.float32 if fp32 else torch.float16, device=x.device)
+    if workspace is None:
+        n = int(lib.exl3_large_m_workspace_bytes(m, k_in, n_out, bits))
+        if n == 0:
+            raise Exl3Error(EXL3_ERR_UNSUPPORTED, "exl3_large_m_workspace_bytes")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=x.device)
+    st = lib.exl3_gemm_large_m(m, _ptr(x), _ptr(packed), _ptr(scale), _ptr(su), _ptr(sv), _ptr(out), int(fp32),
+                               k_in, n_out, bits, _ptr(workspace), workspace.numel() * workspace.element_size(),
+                               _stream(stream))
+    _check(st, "exl3_gemm_large_m")
+    return out
 

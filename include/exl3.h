@@ -163,6 +163,27 @@ EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
                       void *workspace, size_t ws_bytes, void *stream);
 
 /*
+ * exl3_gemm_large_m -- the same product for many input rows (prompt prefill;
+ * the orcasaq2-rocm README reports prefill speeds next to its decode table):
+ * the matrix is decoded once per call into the tensor-core operand layout in
+ * the workspace, then multiplied on the tensor cores (tcgen05).
+ *   m : 1 .. 2^20 rows (efficient from about a hundred; below 32 prefer
+ *       exl3_gemm_small_m, which never materialises the decoded matrix).
+ *   x : m x k_in fp16, row-major.   y : m x n_out (fp16 or fp32), row-major.
+ *   Other arguments as exl3_gemm_small_m, except the workspace:
+ *   workspace, ws_bytes : at least exl3_large_m_workspace_bytes(m, k_in,
+ *     n_out, bits) bytes (2 bytes per weight plus 2 bytes per rotated input
+ *     element, rounded up to the row tile), 256-byte aligned; its first word
+ *     is the status word exl3_workspace_status reads.  No zero-fill needed.
+ * Each output is one accumulator's fixed-order sum: repeated calls are
+ * bitwise identical.
+ */
+EXL3_API size_t exl3_large_m_workspace_bytes(int m, int k_in, int n_out, int bits);
+EXL3_API int exl3_gemm_large_m(int m, const uint16_t *x, const uint32_t *packed, const uint16_t *scale,
+                               const uint16_t *su, const uint16_t *sv, void *y, int y_fp32, int k_in, int n_out,
+                               int bits, void *workspace, size_t ws_bytes, void *stream);
+
+/*
  * exl3_gemm_siblings -- the product for a group of matrices that take the
  * same input: y_i = sv_i .* H(scale_i .* (H(su .* x) W_i)) for i < n_mats,
  * in one pass that rotates x once and spreads all the groups' output blocks

@@ -126,3 +126,22 @@ def test_siblings_validation(ex):
     need = ex.workspace_bytes(32, 256, 512, 3)
     assert call(32, mats(256, 256), 2, wsb=need - 1) == ex.EXL3_ERR_WORKSPACE
     assert call(1, mats(256, 256), 2, ws=16) == ex.EXL3_ERR_MISALIGNED
+
+
+def test_large_m_validation(ex):
+    f = ex.lib.exl3_gemm_large_m
+    need = ex.lib.exl3_large_m_workspace_bytes(300, 256, 256, 3)
+    assert need >= 256 * 256 * 2 + 300 * 256 * 2
+    assert ex.lib.exl3_large_m_workspace_bytes(0, 256, 256, 3) == 0
+    assert ex.lib.exl3_large_m_workspace_bytes(300, 200, 256, 3) == 0
+    args = lambda m=300, k=256, n=256, bits=3, x=16, ws=256, wsb=need: (
+        m, P(x), P(16), P(16), P(16), P(16), P(16), 0, k, n, bits, P(ws), wsb, None)
+    assert f(*args(m=0)) == ex.EXL3_ERR_INVALID_ARG
+    assert f(*args(x=0)) == ex.EXL3_ERR_INVALID_ARG
+    assert f(*args(m=(1 << 20) + 1)) == ex.EXL3_ERR_UNSUPPORTED
+    assert f(*args(k=200)) == ex.EXL3_ERR_UNSUPPORTED
+    assert f(*args(bits=1)) == ex.EXL3_ERR_UNSUPPORTED
+    assert f(*args(x=8)) == ex.EXL3_ERR_MISALIGNED
+    assert f(*args(wsb=need - 1)) == ex.EXL3_ERR_WORKSPACE
+    assert f(*args(ws=0)) == ex.EXL3_ERR_WORKSPACE
+    assert f(*args(ws=16)) == ex.EXL3_ERR_MISALIGNED
