@@ -1,7 +1,6 @@
 // api.cu -- the extern "C" entry points of libexl3 (declared in include/exl3.h):
 // argument validation on the host, architecture check, dispatch to kernels.
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -72,20 +71,8 @@ exl3::GemmArgs single_args(int m, const uint16_t* x, const uint32_t* packed, con
     return a;
 }
 
-// experiment switch (temporary): 0 default, 1 tensor-memory kernel for m >= 2, 2 for every m
-int path_choice()
-{
-    static int v = [] {
-        const char* e = getenv("EXL3_PATH");
-        return e ? atoi(e) : 0;
-    }();
-    return v;
-}
-
 cudaError_t launch_product(const exl3::GemmArgs& a, cudaStream_t s)
 {
-    const int pc = path_choice();
-    if (pc == 2 || (pc == 1 && a.m > 1)) return exl3::launch_gemm_tm(a, s);
     return a.m == 1 ? exl3::launch_gemv_m1(a, s) : exl3::launch_gemm_tc(a, s);
 }
 
@@ -128,9 +115,7 @@ int exl3_version(void) { return 100; }
 size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
     if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
-    const size_t w0 = m == 1 ? exl3::m1_workspace_bytes(k_in, n_out, bits) : exl3::tc_workspace_bytes(m, k_in, n_out, bits);
-    const size_t w1 = exl3::tm_workspace_bytes(m, k_in, n_out, bits);
-    return w0 > w1 ? w0 : w1;
+    return m == 1 ? exl3::m1_workspace_bytes(k_in, n_out, bits) : exl3::tc_workspace_bytes(m, k_in, n_out, bits);
 }
 
 int exl3_kernel_launches(int m, int k_in, int n_out, int bits)

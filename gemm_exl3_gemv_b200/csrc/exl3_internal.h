@@ -91,11 +91,6 @@ int tc_ctas(int m, int k_in, int n_out, int bits);
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
 
-// Tensor-memory path (gemm_tm.cu): decoded 3INST words written to tensor
-// memory as the MMA's A operand.  Workspace size, launcher (two launches).
-size_t tm_workspace_bytes(int m, int k_in, int n_out, int bits);
-cudaError_t launch_gemm_tm(const GemmArgs& a, cudaStream_t stream);
-
 // Many-row path (gemm_large.cu): decode once into the tensor-core operand
 // image, then a tcgen05 GEMM.  Rows per tile (256, 128 or 64: the largest that
 // still gives kLargeMinCtas tiles), workspace size, launcher (three launches).

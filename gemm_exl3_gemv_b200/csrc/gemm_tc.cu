@@ -21,10 +21,11 @@
 //     warp reads the tile row's 256*K contiguous bytes).  The two fp16 halves
 //     of each 3INST word are added once (RNE: the exact decoded weight) and
 //     stored into the warp's own A stage (128 channels x 16 k, MN-major,
-//     128-byte swizzle).  Lane 0 of the warp then issues the MMA itself --
-//     tcgen05.mma kind::f16, M = 128 channels, N = NT rows, K = 16 -- into the
-//     warp's own tensor-memory accumulator (so the accumulation order is
-//     fixed), and commits it to the stage's barrier.  A warp waits only for
+//     128-byte swizzle).  The warp then issues the MMA itself (one elected
+//     lane, from converged code) -- tcgen05.mma kind::f16, M = 128 channels,
+//     N = NT rows, K = 16 -- into the warp's own tensor-memory accumulator
+//     (so the accumulation order is fixed), and commits it to the stage's
+//     barrier.  A warp waits only for
 //     its own stage (two units back) and for the unit's xt.
 //   * A ninth warp streams each unit's xt (1-D bulk copies + mbarrier) into a
 //     four-stage ring shared by the eight decoders.
@@ -343,16 +344,16 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 });
                 fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
-                if (lane == 0) {
-                    if (wait_or_abort(&bfull[bs], bph, abort_flag)) {
-                        tc_fence_after();
-                        const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
-                        mma_f16_ss(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
-                        mma_commit(&aempty[warp * kAStages + s]);
-                        mma_commit(&bempty[bs]);
-                    } else {
-                        fail0 = true;                    // seen by the whole warp at its next unit
-                    }
+                int okb = 1;
+                if (lane == 0) okb = wait_or_abort(&bfull[bs], bph, abort_flag) ? 1 : 0;
+                if (__shfl_sync(0xffffffffu, okb, 0)) {
+                    tc_fence_after();
+                    const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
+                    mma_f16_ss_elect(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
+                    mma_commit_elect(&aempty[warp * kAStages + s]);
+                    mma_commit_elect(&bempty[bs]);
+                } else if (lane == 0) {
+                    fail0 = true;                        // seen by the whole warp at its next unit
                 }
             };
             uint32_t wa[QW], wb[QW];
@@ -368,10 +369,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             if (k < nseg) unit(wa, k, kk + k);
             kk += nseg;
             ok = __shfl_sync(0xffffffffu, (ok && !fail0) ? 1 : 0, 0) != 0;
-            if (lane == 0) {
-                if (ok) mma_commit(segdone);             // arrives once this warp's MMAs are done
-                else mbar_arrive(segdone);
-            }
+            if (ok) mma_commit_elect(segdone);           // arrives once this warp's MMAs are done
+            else if (lane == 0) mbar_arrive(segdone);
 
             // ---- accumulators -> zsm[NT][128] (the eight summed in a fixed order) ----
             int okd = 1;
