@@ -544,14 +544,22 @@ struct TcPlan {
 // Pick the cut of the units for this shape: cost in unit-decode times of the
 // busiest CTA, plus the reduction (stream-K: the last CTA reads every partial
 // of its block, about 0.3 unit-times each; cluster: one pass over shared
-// memory).  A cluster size is used only if all G clusters fit at once.
+// memory), plus kSegCost per segment (the accumulator read-out and partial
+// exchange that ends each block share: a stream-K range crosses block
+// boundaries, a cluster CTA has one segment).  kSegCost = 3 unit-times fits
+// the measured B200 times at M = 32 (5120 -> 17408: clusters of 2, 39.4 us,
+// beat stream-K, 43.3 us; 17408 -> 5120: stream-K, 43.6 us, beats clusters
+// of 6, 44.2 us).  A cluster size is used only if all G clusters fit at once.
+constexpr double kSegCost = 3.0;
 TcPlan choose_plan(int k_in, int n_out, size_t smem)
 {
     auto kern = cluster_fit_probe_kernel;
     const int G = n_out / 128, C = k_in / 128;
     const long long U = (long long)G * C;
     TcPlan sk{0, sk_ctas(k_in, n_out)};
-    const double cost_sk = (double)((U + sk.P - 1) / sk.P) + 0.3 * (double)sk.P / G;
+    const long long per_cta = (U + sk.P - 1) / sk.P;
+    const double segs_sk = 1.0 + (double)(per_cta - 1) / C;      // expected block boundaries crossed, + 1
+    const double cost_sk = (double)per_cta + 0.3 * (double)sk.P / G + kSegCost * segs_sk;
     int Smax = (kSms * kCtasPerSm) / G;
     if (Smax > 10) Smax = 10;          // measured: 16-CTA clusters were slower than 10 (k/v shapes)
     if (Smax > C) Smax = C;
@@ -573,7 +581,7 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
             continue;
         }
         if (nclusters >= G) {
-            const double cost_cl = (double)((C + S - 1) / S) + 0.2 + 0.05 * S;
+            const double cost_cl = (double)((C + S - 1) / S) + 0.2 + 0.05 * S + kSegCost;
             if (cost_cl < cost_sk) return TcPlan{S, G * S};
             break;
         }
