@@ -541,25 +541,44 @@ struct TcPlan {
     int P;   // CTAs launched
 };
 
-// Pick the cut of the units for this shape: cost in unit-decode times of the
-// busiest CTA, plus the reduction (stream-K: the last CTA reads every partial
-// of its block, about 0.3 unit-times each; cluster: one pass over shared
-// memory), plus kSegCost per segment (the accumulator read-out and partial
-// exchange that ends each block share: a stream-K range crosses block
-// boundaries, a cluster CTA has one segment).  kSegCost = 3 unit-times fits
-// the measured B200 times at M = 32 (5120 -> 17408: clusters of 2, 39.4 us,
-// beat stream-K, 43.3 us; 17408 -> 5120: stream-K, 43.6 us, beats clusters
-// of 6, 44.2 us).  A cluster size is used only if all G clusters fit at once.
+// Pick the cut of the units for this shape.  Cost, in unit-decode times, of
+// the busiest CTA:
+//   * its units;
+//   * kSegCost per segment (the accumulator read-out and partial exchange that
+//     ends each block share).  The busiest CTA of an unaligned stream-K cut
+//     has two segments, because ranges straddle blocks; an aligned cut (P a
+//     multiple of G) or a cluster has one;
+//   * the reduction.  Stream-K: the finishing CTA reads P/G partials, about
+//     0.3 unit-times each, plus kGlobalRed for going through global memory.
+//     Cluster: one pass over distributed shared memory.
+// The constants fit measured B200 times at M = 32:
+//   * 5120 -> 17408: clusters of 2, 39.4 us; aligned stream-K, 41.3 us;
+//     stream-K over 296 CTAs, 43.4 us;
+//   * 17408 -> 5120: aligned stream-K over 280 CTAs, 42.3 us; stream-K over
+//     296 CTAs, 43.6 us; clusters of 6, 44.2 us.
+// A cluster size is used only if all G clusters fit at once.
 constexpr double kSegCost = 3.0;
+constexpr double kGlobalRed = 1.2;
 TcPlan choose_plan(int k_in, int n_out, size_t smem)
 {
     auto kern = cluster_fit_probe_kernel;
     const int G = n_out / 128, C = k_in / 128;
     const long long U = (long long)G * C;
-    TcPlan sk{0, sk_ctas(k_in, n_out)};
-    const long long per_cta = (U + sk.P - 1) / sk.P;
-    const double segs_sk = 1.0 + (double)(per_cta - 1) / C;      // expected block boundaries crossed, + 1
-    const double cost_sk = (double)per_cta + 0.3 * (double)sk.P / G + kSegCost * segs_sk;
+    auto cost_sk = [&](long long P) {
+        const long long per = (U + P - 1) / P;
+        const double segs = (P % G == 0) ? 1.0 : (double)((per - 1) / C + 2);
+        return (double)per + 0.3 * (double)P / G + kSegCost * segs + kGlobalRed;
+    };
+    TcPlan best{0, sk_ctas(k_in, n_out)};
+    double best_cost = cost_sk(best.P);
+    // aligned stream-K: S' CTAs per block (S' <= 8 keeps P within the workspace's partial slots)
+    for (int s2 = 2; s2 <= 8 && (long long)s2 * G <= (long long)kSms * kCtasPerSm && s2 <= C; ++s2) {
+        const double c = cost_sk((long long)s2 * G);
+        if (c < best_cost) {
+            best_cost = c;
+            best = TcPlan{0, s2 * G};
+        }
+    }
     int Smax = (kSms * kCtasPerSm) / G;
     if (Smax > 10) Smax = 10;          // measured: 16-CTA clusters were slower than 10 (k/v shapes)
     if (Smax > C) Smax = C;
@@ -582,11 +601,11 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
         }
         if (nclusters >= G) {
             const double cost_cl = (double)((C + S - 1) / S) + 0.2 + 0.05 * S + kSegCost;
-            if (cost_cl < cost_sk) return TcPlan{S, G * S};
+            if (cost_cl < best_cost) best = TcPlan{S, G * S};
             break;
         }
     }
-    return sk;
+    return best;
 }
 
 template <int BITS, int NT>
