@@ -16,7 +16,7 @@
 //      xt (j, c) = NB rows x 64 k = NB * 128 contiguous bytes, rows past m zero.
 //   3. gemm_large_kernel<NB>: CTA (g, j) computes output channels of block g for
 //      rows of tile j.  Warp 0 streams A and B chunks with 1-D bulk copies
-//      (cp.async.bulk + mbarrier) into a 3-stage ring; one thread of warp 1
+//      (cp.async.bulk + mbarrier) into a 3- or 4-stage ring; one thread of warp 1
 //      issues tcgen05.mma kind::f16 (M = 128 channels, N = NB rows, K = 16;
 //      four per 64-row chunk) into one tensor-memory accumulator; then the four
 //      warps drain it 16 rows at a time (tcgen05.ld), scale, rotate, store y.
@@ -35,7 +35,6 @@ namespace exl3 {
 namespace {
 
 constexpr int kLgThreads = 128;
-constexpr int kLgStages = 3;
 constexpr int kAChunk = 16384;                 // A image of one 64-row chunk of one output block
 constexpr uint64_t kLgWaitNs = 2000000000ull;
 
@@ -153,10 +152,14 @@ template <int NB>
 struct LgLayout {
     static constexpr int BCHUNK = NB * 128;                 // B bytes per 64-row chunk
     static constexpr int STAGE = kAChunk + BCHUNK;
+    // ring depth: a 256-row tile runs one CTA per SM and takes four stages (the
+    // bulk-copy latency of three left the tensor pipe half idle, measured);
+    // smaller tiles run two CTAs per SM with three stages each
+    static constexpr int STAGES = NB == 256 ? 4 : 3;
     static constexpr int off_stage = 0;
-    static constexpr int off_z = off_stage + kLgStages * STAGE;   // z [16][128] fp32
+    static constexpr int off_z = off_stage + STAGES * STAGE;   // z [16][128] fp32
     static constexpr int off_bar = off_z + 16 * 128 * 4;
-    static constexpr int nbar = 2 * kLgStages + 1;          // full[], empty[], done
+    static constexpr int nbar = 2 * STAGES + 1;          // full[], empty[], done
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
     static_assert(STAGE % 1024 == 0 && off_z % 1024 == 0, "layout");
@@ -198,8 +201,8 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-    uint64_t* empty = full + kLgStages;
-    uint64_t* done = empty + kLgStages;
+    uint64_t* empty = full + L::STAGES;
+    uint64_t* done = empty + L::STAGES;
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
@@ -210,7 +213,7 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     const int C64 = prm.k_in / 64;
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kLgStages; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
+        for (int i = 0; i < L::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
         mbar_init(done, 1);
         misc[1] = 0;
         fence_mbar_init();
@@ -231,8 +234,8 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
         const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
         int issued = 0;
         for (int c = 0; c < C64; ++c) {
-            const int s = c % kLgStages;
-            if (c >= kLgStages && !lg_wait(&empty[s], (uint32_t)(c / kLgStages - 1) & 1u, abort_flag)) break;
+            const int s = c % L::STAGES;
+            if (c >= L::STAGES && !lg_wait(&empty[s], (uint32_t)(c / L::STAGES - 1) & 1u, abort_flag)) break;
             mbar_arrive_expect_tx(&full[s], L::STAGE);
             uint8_t* st = smem + L::off_stage + s * L::STAGE;
             bulk_g2s(st, a_src + (size_t)c * kAChunk, kAChunk, &full[s]);
@@ -241,15 +244,15 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
         }
         // on abort, let every issued copy land before the CTA can exit
         if (*abort_flag)
-            for (int v = issued > kLgStages ? issued - kLgStages : 0; v < issued; ++v)
-                (void)mbar_wait_bounded(&full[v % kLgStages], (uint32_t)(v / kLgStages) & 1u, 100000000ull);
+            for (int v = issued > L::STAGES ? issued - L::STAGES : 0; v < issued; ++v)
+                (void)mbar_wait_bounded(&full[v % L::STAGES], (uint32_t)(v / L::STAGES) & 1u, 100000000ull);
     } else if (warp == 1 && lane == 0) {
         // ---- MMA issuer: four K = 16 steps per chunk into the accumulator ----
         constexpr uint32_t idesc = idesc_f16_amn(128, NB);
         bool ok = true;
         for (int c = 0; c < C64 && ok; ++c) {
-            const int s = c % kLgStages;
-            if (!lg_wait(&full[s], (uint32_t)(c / kLgStages) & 1u, abort_flag)) { ok = false; break; }
+            const int s = c % L::STAGES;
+            if (!lg_wait(&full[s], (uint32_t)(c / L::STAGES) & 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             const uint32_t st = smem_u32(smem + L::off_stage + s * L::STAGE);
 #pragma unroll
