@@ -267,6 +267,21 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     __syncwarp();
 
     // ---- epilogue: 16 rows at a time, accumulator -> z -> y ----
+    // this lane's four output channels: scale and signs, the same for every row
+    // (loaded while the last MMAs run)
+    const int n0 = 128 * g + 4 * lane;
+    float osc[4], osg[4];
+    {
+        const uint2 sc = *reinterpret_cast<const uint2*>(prm.scale + n0);
+        const uint2 sg = *reinterpret_cast<const uint2*>(prm.sv + n0);
+        const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+        const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+        const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+        const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+        osc[0] = sc0.x; osc[1] = sc0.y; osc[2] = sc1.x; osc[3] = sc1.y;
+        osg[0] = kInvSqrt128 * sg0.x; osg[1] = kInvSqrt128 * sg0.y;
+        osg[2] = kInvSqrt128 * sg1.x; osg[3] = kInvSqrt128 * sg1.y;
+    }
     int okd = 1;
     if (lane == 0) okd = lg_wait(done, 0u, abort_flag) ? 1 : 0;
     okd = __shfl_sync(0xffffffffu, okd, 0);
@@ -289,20 +304,13 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
         for (int i = 0; i < 4; ++i) {
             const int mm = j * NB + t0 + 4 * warp + i;
             if (mm >= prm.m) break;
-            const int n0 = 128 * g + 4 * lane;
             const float4 z4 = *reinterpret_cast<const float4*>(zsm + (4 * warp + i) * 128 + 4 * lane);
-            const uint2 sc = *reinterpret_cast<const uint2*>(prm.scale + n0);
-            const uint2 sg = *reinterpret_cast<const uint2*>(prm.sv + n0);
-            const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
-            const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
-            const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
-            const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
-            float vv[4] = {z4.x * sc0.x, z4.y * sc0.y, z4.z * sc1.x, z4.w * sc1.y};
+            float vv[4] = {z4.x * osc[0], z4.y * osc[1], z4.z * osc[2], z4.w * osc[3]};
             fwht128_warp(vv);
-            vv[0] *= kInvSqrt128 * sg0.x;
-            vv[1] *= kInvSqrt128 * sg0.y;
-            vv[2] *= kInvSqrt128 * sg1.x;
-            vv[3] *= kInvSqrt128 * sg1.y;
+            vv[0] *= osg[0];
+            vv[1] *= osg[1];
+            vv[2] *= osg[2];
+            vv[3] *= osg[3];
             const size_t yo = (size_t)mm * prm.n_out + n0;
             if (prm.y_fp32) {
                 *reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
