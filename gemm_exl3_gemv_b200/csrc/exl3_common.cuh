@@ -154,6 +154,36 @@ __device__ __forceinline__ void fwht128_warp(float (&v)[4])
     }
 }
 
+// fwht128_warp on R independent rows at once (same arithmetic per row): each
+// shuffle stage issues R*4 independent shuffles, so one warp hides the
+// shuffle latency that a row-by-row loop exposes.
+template <int R>
+__device__ __forceinline__ void fwht128_warp_rows(float (&v)[R][4])
+{
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+        float a0 = v[r][0] + v[r][1], a1 = v[r][0] - v[r][1], a2 = v[r][2] + v[r][3], a3 = v[r][2] - v[r][3];
+        v[r][0] = a0 + a2;
+        v[r][1] = a1 + a3;
+        v[r][2] = a0 - a2;
+        v[r][3] = a1 - a3;
+    }
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const bool upper = (lane & d) != 0;
+        float p[R][4];
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) p[r][e] = __shfl_xor_sync(0xffffffffu, v[r][e], d);
+#pragma unroll
+        for (int r = 0; r < R; ++r)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) v[r][e] = upper ? (p[r][e] - v[r][e]) : (v[r][e] + p[r][e]);
+    }
+}
+
 constexpr float kInvSqrt128 = 0.08838834764831845f;
 
 }  // namespace exl3

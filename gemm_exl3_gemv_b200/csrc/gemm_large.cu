@@ -14,12 +14,15 @@
 //   2. xt_tiled_prepass_kernel: xt = H(su .* x) in fp16, laid out as the B
 //      operand (K-major, 128-byte swizzle) per tile of NB input rows:
 //      xt (j, c) = NB rows x 64 k = NB * 128 contiguous bytes, rows past m zero.
-//   3. gemm_large_kernel<NB>: CTA (g, j) computes output channels of block g for
-//      rows of tile j.  Warp 0 streams A and B chunks with 1-D bulk copies
-//      (cp.async.bulk + mbarrier) into a 3- or 4-stage ring; one thread of warp 1
-//      issues tcgen05.mma kind::f16 (M = 128 channels, N = NB rows, K = 16;
-//      four per 64-row chunk) into one tensor-memory accumulator; then the four
-//      warps drain it 16 rows at a time (tcgen05.ld), scale, rotate, store y.
+//   3. gemm_large_kernel<NB>: persistent CTAs (one wave), each taking every
+//      gridDim-th tile (output block g, row tile j).  Warp 0 streams A and B
+//      chunks with 1-D bulk copies (cp.async.bulk + mbarrier) into a 3- or
+//      4-stage ring that runs on across tiles; one thread of warp 1 issues
+//      tcgen05.mma kind::f16 (M = 128 channels, N = NB rows, K = 16; four per
+//      64-row chunk) into one of two tensor-memory accumulators, alternating
+//      per tile; warps 4-7 drain the other one 16 rows at a time (tcgen05.ld),
+//      scale, rotate and store y -- the epilogue of a tile overlaps the
+//      mainloop of the next.
 //   No split-K: each output element is one accumulator's fixed-order sum, so
 //   results are bitwise repeatable.  Every wait is bounded (2 s).
 #include <atomic>
@@ -34,7 +37,8 @@ namespace exl3 {
 
 namespace {
 
-constexpr int kLgThreads = 128;
+constexpr int kLgThreads = 256;                // warp 0 producer, warp 1 MMA issuer, warps 4-7 epilogue
+constexpr int kLgEpiWarp0 = 4;
 constexpr int kAChunk = 16384;                 // A image of one 64-row chunk of one output block
 constexpr uint64_t kLgWaitNs = 2000000000ull;
 
@@ -159,14 +163,20 @@ struct LgLayout {
     static constexpr int off_stage = 0;
     static constexpr int off_z = off_stage + STAGES * STAGE;   // z [16][128] fp32
     static constexpr int off_bar = off_z + 16 * 128 * 4;
-    static constexpr int nbar = 2 * STAGES + 1;          // full[], empty[], done
+    // full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], last
+    static constexpr int nbar = 2 * STAGES + 5;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;      // + slack to align the base to 1024
+    // two accumulators of NB columns (the epilogue of one tile overlaps the
+    // mainloop of the next); CTAS_PER_SM resident CTAs fill tensor memory exactly
+    static constexpr int TMEM_COLS = 2 * NB;
+    static constexpr int CTAS_PER_SM = NB == 256 ? 1 : 2;
     static_assert(STAGE % 1024 == 0 && off_z % 1024 == 0, "layout");
     static_assert(total <= 227 * 1024, "shared memory");
-    // NB <= 256 columns of tensor memory; with at most two CTAs of this size
-    // per SM (shared memory), allocations never wait
     static_assert(NB == 64 || NB == 128 || NB == 256, "tensor memory columns");
+    static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "tensor memory");
+    // no further CTA fits on an SM (shared memory), so allocations never wait
+    static_assert((CTAS_PER_SM + 1) * (total + 1024) > 228 * 1024, "CTAs per SM");
 };
 
 struct LgParams {
@@ -177,6 +187,7 @@ struct LgParams {
     void* y;
     uint32_t* status;
     int y_fp32, m, k_in, n_out;
+    int J;                    // row tiles (m_pad / NB)
 };
 
 __device__ __forceinline__ bool lg_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
@@ -202,24 +213,27 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::off_bar);
     uint64_t* empty = full + L::STAGES;
-    uint64_t* done = empty + L::STAGES;
+    uint64_t* acc_full = empty + L::STAGES;      // [2]: the tile's MMAs into accumulator a completed
+    uint64_t* acc_empty = acc_full + 2;          // [2]: the epilogue has read accumulator a
+    uint64_t* lastbar = acc_empty + 2;           // every MMA of the CTA completed
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = prm.n_out / 128;
-    const int g = blockIdx.x % G, j = blockIdx.x / G;
+    const int tiles = G * prm.J;                 // tile t: output block t % G, row tile t / G
     const int C64 = prm.k_in / 64;
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < L::STAGES; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-        mbar_init(done, 1);
+        for (int i = 0; i < 2; ++i) { mbar_init(&acc_full[i], 1); mbar_init(&acc_empty[i], 4); }
+        mbar_init(lastbar, 1);
         misc[1] = 0;
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), NB);
+        tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), L::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -229,97 +243,129 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     grid_dep_wait();                                   // A and B images are the pre-passes' output
 
     if (warp == 0 && lane == 0) {
-        // ---- producer: A and B chunks of this tile into the stage ring ----
-        const uint8_t* a_src = prm.image + (size_t)g * C64 * kAChunk;
-        const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
-        int issued = 0;
-        for (int c = 0; c < C64; ++c) {
-            const int s = c % L::STAGES;
-            if (c >= L::STAGES && !lg_wait(&empty[s], (uint32_t)(c / L::STAGES - 1) & 1u, abort_flag)) break;
-            mbar_arrive_expect_tx(&full[s], L::STAGE);
-            uint8_t* st = smem + L::off_stage + s * L::STAGE;
-            bulk_g2s(st, a_src + (size_t)c * kAChunk, kAChunk, &full[s]);
-            bulk_g2s(st + kAChunk, b_src + (size_t)c * L::BCHUNK, L::BCHUNK, &full[s]);
-            issued = c + 1;
+        // ---- producer: A and B chunks of this CTA's tiles into the stage ring ----
+        int q = 0;                                     // chunks issued (ring position)
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
+            const int g = t % G, j = t / G;
+            const uint8_t* a_src = prm.image + (size_t)g * C64 * kAChunk;
+            const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
+            for (int c = 0; c < C64; ++c, ++q) {
+                const int s = q % L::STAGES;
+                if (q >= L::STAGES && !lg_wait(&empty[s], (uint32_t)(q / L::STAGES - 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&full[s], L::STAGE);
+                uint8_t* st = smem + L::off_stage + s * L::STAGE;
+                bulk_g2s(st, a_src + (size_t)c * kAChunk, kAChunk, &full[s]);
+                bulk_g2s(st + kAChunk, b_src + (size_t)c * L::BCHUNK, L::BCHUNK, &full[s]);
+            }
         }
         // on abort, let every issued copy land before the CTA can exit
         if (*abort_flag)
-            for (int v = issued > L::STAGES ? issued - L::STAGES : 0; v < issued; ++v)
+            for (int v = q > L::STAGES ? q - L::STAGES : 0; v < q; ++v)
                 (void)mbar_wait_bounded(&full[v % L::STAGES], (uint32_t)(v / L::STAGES) & 1u, 100000000ull);
     } else if (warp == 1 && lane == 0) {
-        // ---- MMA issuer: four K = 16 steps per chunk into the accumulator ----
+        // ---- MMA issuer: per tile, four K = 16 steps per chunk into accumulator it & 1 ----
         constexpr uint32_t idesc = idesc_f16_amn(128, NB);
         bool ok = true;
-        for (int c = 0; c < C64 && ok; ++c) {
-            const int s = c % L::STAGES;
-            if (!lg_wait(&full[s], (uint32_t)(c / L::STAGES) & 1u, abort_flag)) { ok = false; break; }
-            tc_fence_after();
-            const uint32_t st = smem_u32(smem + L::off_stage + s * L::STAGE);
-#pragma unroll
-            for (int t = 0; t < 4; ++t)
-                mma_f16_ss(tmem, sdesc_sw128(st + t * 4096, 1024, 2048), sdesc_sw128(st + kAChunk + t * 32, 16, 1024),
-                           idesc, (c > 0 || t > 0) ? 1u : 0u);
-            mma_commit(&empty[s]);
-        }
-        if (ok) mma_commit(done);
-        else mbar_arrive(done);
-    }
-    __syncwarp();
-
-    // ---- epilogue: 16 rows at a time, accumulator -> z -> y ----
-    // this lane's four output channels: scale and signs, the same for every row
-    // (loaded while the last MMAs run)
-    const int n0 = 128 * g + 4 * lane;
-    float osc[4], osg[4];
-    {
-        const uint2 sc = *reinterpret_cast<const uint2*>(prm.scale + n0);
-        const uint2 sg = *reinterpret_cast<const uint2*>(prm.sv + n0);
-        const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
-        const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
-        const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
-        const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
-        osc[0] = sc0.x; osc[1] = sc0.y; osc[2] = sc1.x; osc[3] = sc1.y;
-        osg[0] = kInvSqrt128 * sg0.x; osg[1] = kInvSqrt128 * sg0.y;
-        osg[2] = kInvSqrt128 * sg1.x; osg[3] = kInvSqrt128 * sg1.y;
-    }
-    int okd = 1;
-    if (lane == 0) okd = lg_wait(done, 0u, abort_flag) ? 1 : 0;
-    okd = __shfl_sync(0xffffffffu, okd, 0);
-    tc_fence_after();
-    const int ch = chan_of_row(32 * warp + lane);
-    for (int t0 = 0; t0 < NB; t0 += 16) {
-        if (j * NB + t0 >= prm.m) break;                  // uniform: rows past m are padding
-        uint32_t t16[16];
-        if (okd) {
-            tmem_ld16(tmem + ((uint32_t)(32 * warp) << 16) + (uint32_t)t0, t16);
-            tmem_ld_wait();
-        } else {
-#pragma unroll
-            for (int t = 0; t < 16; ++t) t16[t] = 0u;
-        }
-#pragma unroll
-        for (int t = 0; t < 16; ++t) zsm[t * 128 + ch] = __uint_as_float(t16[t]);
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int mm = j * NB + t0 + 4 * warp + i;
-            if (mm >= prm.m) break;
-            const float4 z4 = *reinterpret_cast<const float4*>(zsm + (4 * warp + i) * 128 + 4 * lane);
-            float vv[4] = {z4.x * osc[0], z4.y * osc[1], z4.z * osc[2], z4.w * osc[3]};
-            fwht128_warp(vv);
-            vv[0] *= osg[0];
-            vv[1] *= osg[1];
-            vv[2] *= osg[2];
-            vv[3] *= osg[3];
-            const size_t yo = (size_t)mm * prm.n_out + n0;
-            if (prm.y_fp32) {
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.y) + yo) = make_float4(vv[0], vv[1], vv[2], vv[3]);
-            } else {
-                __half2 hh[2] = {__floats2half2_rn(vv[0], vv[1]), __floats2half2_rn(vv[2], vv[3])};
-                *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(prm.y) + yo) = *reinterpret_cast<uint2*>(hh);
+        int q = 0, it = 0;
+        for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x, ++it) {
+            const int acc = it & 1;
+            const uint32_t d = tmem + (uint32_t)(acc * NB);
+            if (it >= 2 && !lg_wait(&acc_empty[acc], (uint32_t)((it >> 1) - 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
             }
+            tc_fence_after();
+            for (int c = 0; c < C64; ++c, ++q) {
+                const int s = q % L::STAGES;
+                if (!lg_wait(&full[s], (uint32_t)(q / L::STAGES) & 1u, abort_flag)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t st = smem_u32(smem + L::off_stage + s * L::STAGE);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_f16_ss(d, sdesc_sw128(st + k * 4096, 1024, 2048), sdesc_sw128(st + kAChunk + k * 32, 16, 1024),
+                               idesc, (c > 0 || k > 0) ? 1u : 0u);
+                mma_commit(&empty[s]);
+            }
+            if (ok) mma_commit(&acc_full[acc]);
         }
-        __syncthreads();
+        // every MMA issued here completes before the CTA may free tensor memory
+        mma_commit(lastbar);
+        (void)mbar_wait_bounded(lastbar, 0u, 100000000ull);
+    } else if (warp >= kLgEpiWarp0) {
+        // ---- epilogue warps (tensor-memory lanes 32 * (warp % 4)): accumulator -> z -> y,
+        // 16 rows at a time, while the next tile's MMAs run into the other accumulator ----
+        const int ew = warp - kLgEpiWarp0;                         // == warp % 4
+        const int ch = chan_of_row(32 * ew + lane);
+        int it = 0;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
+            const int acc = it & 1, g = t % G, j = t / G;
+            // this lane's four output channels of block g: scale and signs
+            const int n0 = 128 * g + 4 * lane;
+            float osc[4], osg[4];
+            {
+                const uint2 sc = *reinterpret_cast<const uint2*>(prm.scale + n0);
+                const uint2 sg = *reinterpret_cast<const uint2*>(prm.sv + n0);
+                const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
+                const float2 sc1 = __half22float2(*reinterpret_cast<const __half2*>(&sc.y));
+                const float2 sg0 = __half22float2(*reinterpret_cast<const __half2*>(&sg.x));
+                const float2 sg1 = __half22float2(*reinterpret_cast<const __half2*>(&sg.y));
+                osc[0] = sc0.x; osc[1] = sc0.y; osc[2] = sc1.x; osc[3] = sc1.y;
+                osg[0] = kInvSqrt128 * sg0.x; osg[1] = kInvSqrt128 * sg0.y;
+                osg[2] = kInvSqrt128 * sg1.x; osg[3] = kInvSqrt128 * sg1.y;
+            }
+            int okd = 1;
+            if (lane == 0) okd = lg_wait(&acc_full[acc], (uint32_t)(it >> 1) & 1u, abort_flag) ? 1 : 0;
+            okd = __shfl_sync(0xffffffffu, okd, 0);
+            tc_fence_after();
+            for (int t0 = 0; t0 < NB; t0 += 16) {
+                if (j * NB + t0 >= prm.m) break;              // uniform: rows past m are padding
+                uint32_t t16[16];
+                if (okd) {
+                    tmem_ld16(tmem + ((uint32_t)(32 * ew) << 16) + (uint32_t)(acc * NB + t0), t16);
+                    tmem_ld_wait();
+                } else {
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) t16[u] = 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 16; ++u) zsm[u * 128 + ch] = __uint_as_float(t16[u]);
+                named_bar(1, 128);
+                // this warp's four rows together (independent shuffle chains)
+                float vv[4][4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float4 z4 = *reinterpret_cast<const float4*>(zsm + (4 * ew + i) * 128 + 4 * lane);
+                    vv[i][0] = z4.x * osc[0];
+                    vv[i][1] = z4.y * osc[1];
+                    vv[i][2] = z4.z * osc[2];
+                    vv[i][3] = z4.w * osc[3];
+                }
+                fwht128_warp_rows<4>(vv);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int mm = j * NB + t0 + 4 * ew + i;
+                    if (mm >= prm.m) break;
+                    const size_t yo = (size_t)mm * prm.n_out + n0;
+                    const float o0 = vv[i][0] * osg[0], o1 = vv[i][1] * osg[1];
+                    const float o2 = vv[i][2] * osg[2], o3 = vv[i][3] * osg[3];
+                    if (prm.y_fp32) {
+                        *reinterpret_cast<float4*>(reinterpret_cast<float*>(prm.y) + yo) = make_float4(o0, o1, o2, o3);
+                    } else {
+                        __half2 hh[2] = {__floats2half2_rn(o0, o1), __floats2half2_rn(o2, o3)};
+                        *reinterpret_cast<uint2*>(reinterpret_cast<__half*>(prm.y) + yo) = *reinterpret_cast<uint2*>(hh);
+                    }
+                }
+                named_bar(1, 128);
+            }
+            // accumulator read out: the MMA issuer may reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
     }
     grid_dep_launch();
 
@@ -328,7 +374,7 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, NB);
+        tmem_dealloc(tmem, L::TMEM_COLS);
     }
     if (threadIdx.x == 0 && misc[1]) atomicOr(prm.status, kStatusTimeout);
 }
@@ -365,12 +411,20 @@ cudaError_t launch_gemm_large_nb(const LgParams& prm, cudaStream_t stream, int p
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
     });
     if (e != cudaSuccess) return e;
-    const int G = prm.n_out / 128, J = (prm.m + NB - 1) / NB;
+    const int G = prm.n_out / 128;
+    // persistent: at most one wave of resident CTAs, each taking every gridDim-th tile
+    int sms = 0, dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const long long tiles = (long long)G * prm.J;
+    const long long slots = (long long)sms * L::CTAS_PER_SM;
+    const int grid = (int)(tiles < slots ? tiles : slots);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3((unsigned)(G * J), 1, 1);
+    cfg.gridDim = dim3((unsigned)grid, 1, 1);
     cfg.blockDim = dim3(kLgThreads, 1, 1);
     cfg.dynamicSmemBytes = L::total;
     cfg.stream = stream;
@@ -439,6 +493,7 @@ cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
     prm.m = a.m;
     prm.k_in = a.k_in;
     prm.n_out = a.n_out;
+    prm.J = m_pad / nb;
     switch (nb) {
         case 256: e = launch_gemm_large_nb<256>(prm, stream, a.pdl); break;
         case 128: e = launch_gemm_large_nb<128>(prm, stream, a.pdl); break;
