@@ -43,7 +43,9 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--m", type=int, default=32)
+    ap.add_argument("--m", type=int, default=32,
+                    help="input rows; above 32 the products go through the many-row (prefill) call, "
+                         "with the synthetic rows repeated to m")
     ap.add_argument("--layers", type=int, default=64)
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -96,6 +98,17 @@ def load_peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def load_tensor_peak():
+    """Dense fp16/bf16 tensor peak (the same nominal rate for both), burst."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured (bf16 burst)"
+    return 1590.0, "fallback"
 
 
 # --------------------------------------------------------------- clocks ----
@@ -244,8 +257,11 @@ class Stack:
         self.y_dev = torch.empty(yo, dtype=torch.float16, device=device)
         self.x_pin = torch.empty(xo, dtype=torch.float16).pin_memory()
         self.y_pin = torch.empty(yo, dtype=torch.float16).pin_memory()
+        self.large = m > 32
         for i, (spec, packed) in enumerate(zip(specs, weights)):
             scale, x, su, sv = synth.small_inputs(spec)
+            if x.shape[0] < m:                          # many-row runs: the synthetic rows repeated
+                x = np.tile(x, ((m + x.shape[0] - 1) // x.shape[0], 1))
             t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
             xs = slice(x_off[i], x_off[i] + m * spec.k_in)
             ys = slice(y_off[i], y_off[i] + m * spec.n_out)
@@ -253,7 +269,8 @@ class Stack:
             self.x_dev[xs].copy_(self.x_pin[xs])
             self.mats.append({"spec": spec, "packed": packed, "scale": t(scale), "su": t(su), "sv": t(sv),
                               "x": self.x_dev[xs].view(m, spec.k_in), "y": self.y_dev[ys].view(m, spec.n_out)})
-            ws_need = max(ws_need, ex.workspace_bytes(m, spec.k_in, spec.n_out, spec.bits))
+            ws_need = max(ws_need, int(ex.lib.exl3_large_m_workspace_bytes(m, spec.k_in, spec.n_out, spec.bits))
+                          if self.large else ex.workspace_bytes(m, spec.k_in, spec.n_out, spec.bits))
         # per layer: its matrices and its contiguous x and y slices
         self.layers = []
         for i, spec in enumerate(specs):
@@ -268,16 +285,19 @@ class Stack:
         self.ws = torch.zeros(ws_need, dtype=torch.uint8, device=device)
         self.ex = ex
         self.packed_bytes = sum(s.packed_bytes for s in self.specs)
-        self.launches = sum(ex.kernel_launches(m, s.k_in, s.n_out, s.bits) for s in self.specs)
+        # the many-row call launches three kernels (decode image, input rotation, GEMM)
+        self.launches = sum(3 if self.large else ex.kernel_launches(m, s.k_in, s.n_out, s.bits)
+                            for s in self.specs)
         self.io_bytes = sum(2 * m * (s.k_in + s.n_out) + 2 * (s.k_in + 2 * s.n_out) for s in self.specs)
         self.h2d = self.x_pin.numel() * 2
         self.d2h = self.y_pin.numel() * 2
 
     def run_mats(self, mats):
         ex = self.ex
+        call = ex.gemm_large if self.large else ex.gemm
         for mt in mats:
-            ex.gemm(mt["x"], mt["packed"], mt["scale"], mt["su"], mt["sv"], mt["spec"].bits, out=mt["y"],
-                    workspace=self.ws)
+            call(mt["x"], mt["packed"], mt["scale"], mt["su"], mt["sv"], mt["spec"].bits, out=mt["y"],
+                 workspace=self.ws)
 
     def run(self):
         self.run_mats(self.mats)
@@ -403,7 +423,7 @@ def run_ours(args, world, rank, local):
     peak, peak_kind = load_peaks()
     algo_bytes = st.packed_bytes + st.io_bytes
     achieved = algo_bytes / (main["ms"] * 1e-3) / 1e9
-    ratio, traffic_src = measured_traffic_ratio() if args.m > 1 else (None, None)
+    ratio, traffic_src = measured_traffic_ratio() if 1 < args.m <= 32 else (None, None)
     traffic = round(ratio * st.packed_bytes / len(st.specs)) if ratio else None
     line = {
         "metric": METRIC, "value": round(gbs * world, 3), "unit": UNIT, "n_gpus": world,
@@ -432,6 +452,17 @@ def run_ours(args, world, rank, local):
                      "traffic_source": traffic_src,
                      "launches_per_step": st.launches},
     }
+    if st.large:
+        # many rows: a dense contraction on the tensor cores (fp16 in, fp32 accumulate)
+        flops = sum(2.0 * args.m * s.k_in * s.n_out for s in st.specs)
+        tflops = flops / (main["ms"] * 1e-3) / 1e12
+        tpeak, tkind = load_tensor_peak()
+        line["tflops"] = round(tflops, 1)
+        line["roofline"] = {"bound": "tensor", "achieved": round(tflops, 1), "peak": tpeak, "unit": "TFLOP/s",
+                            "frac": round(tflops / tpeak, 4), "traffic": None, "peak_kind": tkind,
+                            "kernel": "many-row product (decode image + input rotation + tcgen05 GEMM), "
+                                      "2 m k n flops per product / (CUDA-event step time / products)",
+                            "traffic_source": None, "launches_per_step": st.launches}
     if 1 in results and args.m != 1:
         r1 = results[1]
         line["us_per_layer_m1"] = round(r1["ms"] * 1e3 / layers, 3)

@@ -188,6 +188,7 @@ struct LgParams {
     uint32_t* status;
     int y_fp32, m, k_in, n_out;
     int J;                    // row tiles (m_pad / NB)
+    int jfast;                // tile order: 1 = row tile fastest, 0 = output block fastest
 };
 
 __device__ __forceinline__ bool lg_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag)
@@ -202,6 +203,22 @@ __device__ __forceinline__ bool lg_wait(uint64_t* bar, uint32_t parity, volatile
             atomicExch((int*)abort_flag, 1);
             return false;
         }
+    }
+}
+
+// Tile t of the persistent order.  A wave of resident CTAs covers consecutive
+// tiles, so the order decides what must stay in L2: output-block fastest keeps
+// the whole A image and a few row tiles of xt; row-tile fastest keeps the
+// whole xt and a few output blocks of the image.  The launcher picks the
+// smaller set.
+__device__ __forceinline__ void tile_of(const LgParams& prm, int G, int t, int& g, int& j)
+{
+    if (prm.jfast) {
+        j = t % prm.J;
+        g = t / prm.J;
+    } else {
+        g = t % G;
+        j = t / G;
     }
 }
 
@@ -222,7 +239,7 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = prm.n_out / 128;
-    const int tiles = G * prm.J;                 // tile t: output block t % G, row tile t / G
+    const int tiles = G * prm.J;                 // tile t -> (g, j): see tile_of
     const int C64 = prm.k_in / 64;
 
     if (threadIdx.x == 0) {
@@ -247,7 +264,8 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
         int q = 0;                                     // chunks issued (ring position)
         bool ok = true;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
-            const int g = t % G, j = t / G;
+            int g, j;
+            tile_of(prm, G, t, g, j);
             const uint8_t* a_src = prm.image + (size_t)g * C64 * kAChunk;
             const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
             for (int c = 0; c < C64; ++c, ++q) {
@@ -302,7 +320,9 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
         const int ch = chan_of_row(32 * ew + lane);
         int it = 0;
         for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++it) {
-            const int acc = it & 1, g = t % G, j = t / G;
+            const int acc = it & 1;
+            int g, j;
+            tile_of(prm, G, t, g, j);
             // this lane's four output channels of block g: scale and signs
             const int n0 = 128 * g + 4 * lane;
             float osc[4], osg[4];
@@ -494,6 +514,15 @@ cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
     prm.k_in = a.k_in;
     prm.n_out = a.n_out;
     prm.J = m_pad / nb;
+    {
+        // L2 working set of a wave of tiles in each order (bytes): keep the smaller
+        const double image = 2.0 * a.k_in * a.n_out, xtb = 2.0 * m_pad * a.k_in;
+        const double wave = 148.0;                 // about one tile per SM in flight
+        const double G = a.n_out / 128, J = prm.J;
+        const double g_fast = image + xtb * (wave / G < J ? wave / G : J) / J;
+        const double j_fast = xtb + image * (wave / J < G ? wave / J : G) / G;
+        prm.jfast = j_fast < g_fast ? 1 : 0;
+    }
     switch (nb) {
         case 256: e = launch_gemm_large_nb<256>(prm, stream, a.pdl); break;
         case 128: e = launch_gemm_large_nb<128>(prm, stream, a.pdl); break;
