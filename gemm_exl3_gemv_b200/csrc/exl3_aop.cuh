@@ -7,6 +7,9 @@
 #include <cstdint>
 #include <utility>
 
+#include <cuda_fp16.h>
+
+#include "exl3_common.cuh"
 #include "exl3_decode.cuh"
 
 namespace exl3 {
@@ -67,6 +70,85 @@ __device__ __forceinline__ void lane_soff(int lane, uint32_t (&soff)[2][2])
 #pragma unroll
         for (int e = 0; e < 2; ++e)
             soff[rb][e] = atom * 1024 + (4 * rb + q) * 128 + ((uint32_t)(chunk_of_tile(j4, e) ^ (4 * rb + q)) << 4);
+}
+
+
+// xt = H(su .* x) / sqrt(128) as the MMA's B operand (K-major, 128-byte
+// swizzle), for one warp item (row m, four 128-blocks of K_in): item
+// < m_pad * ceil(K_in / 512).  Rows m_rows .. m_pad - 1 are written as zeros.
+// Layout: per tile of nb rows and 64 k, nb x 128 contiguous bytes; row r of
+// the tile at (r >> 3) * 1024 + (r & 7) * 128, its 16-byte pieces swizzled by
+// (r & 7); inside each 16-row group of k, row k = 4q + s sits at position
+// 4s + q (the A image's order).  One lane takes 16 consecutive inputs (one
+// tile row), loaded and stored 16 bytes at a time; the transform runs over
+// index bits 0-3 in registers and bits 4-6 across the eight lanes of a group.
+__device__ __forceinline__ void xt_rotate_item(const __half* __restrict__ x, const __half* __restrict__ su,
+                                               int m_rows, int k_in, int nb, uint8_t* __restrict__ xt,
+                                               long long item)
+{
+    const int lane = threadIdx.x & 31;
+    const int nblk = k_in / 128, nb4 = (nblk + 3) / 4;
+    const int m = (int)(item / nb4), b = 4 * (int)(item % nb4) + (lane >> 3), l8 = lane & 7;
+    const bool valid = b < nblk;                                // uniform per lane group
+    const int k0 = 128 * b + 16 * l8;
+    float v[16];
+    if (valid && m < m_rows) {
+        const uint4* xp = reinterpret_cast<const uint4*>(x + (size_t)m * k_in + k0);
+        const uint4* sp = reinterpret_cast<const uint4*>(su + k0);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint4 xv = xp[h], sv = sp[h];
+            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w}, sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 xf = __half22float2(*reinterpret_cast<const __half2*>(&xw[t]));
+                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sw[t]));
+                v[8 * h + 2 * t] = xf.x * sf.x;
+                v[8 * h + 2 * t + 1] = xf.y * sf.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = 0.f;
+    }
+#pragma unroll
+    for (int d = 1; d < 16; d <<= 1)                            // index bits 0-3: in registers
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            if ((i & d) == 0) {
+                const float a0 = v[i], a1 = v[i + d];
+                v[i] = a0 + a1;
+                v[i + d] = a0 - a1;
+            }
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) {                           // index bits 4-6: lanes of the group
+        const bool upper = (l8 & d) != 0;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const float p = __shfl_xor_sync(0xffffffffu, v[i], d);
+            v[i] = upper ? (p - v[i]) : (v[i] + p);
+        }
+    }
+    if (valid) {
+        // tile row tr = 8b + l8; inside it, position p holds row k16 = 4(p & 3) + (p >> 2)
+        const int tr = 8 * b + l8;
+        const int kchunk = tr >> 2, c16 = 2 * (tr & 3);
+        const int j = m / nb, mr = m % nb;
+        uint8_t* base = xt + ((size_t)j * (k_in / 64) + kchunk) * nb * 128 + (mr >> 3) * 1024 + (mr & 7) * 128;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            uint32_t o[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const int p0 = 8 * h + 2 * t, p1 = p0 + 1;
+                const float f0 = v[4 * (p0 & 3) + (p0 >> 2)] * kInvSqrt128;
+                const float f1 = v[4 * (p1 & 3) + (p1 >> 2)] * kInvSqrt128;
+                const __half2 hh = __floats2half2_rn(f0, f1);
+                o[t] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            *reinterpret_cast<uint4*>(base + (((c16 + h) ^ (mr & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+    }
 }
 
 }  // namespace exl3
