@@ -195,7 +195,9 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
     if (warp == 0 && lane == 0) {
         // ---- producer: A and B chunks of this CTA's tiles into the stage ring ----
         int q = 0;                                     // chunks issued (ring position)
-        bool ok = true;
+        // a nonzero injection word (tests of the timeout path) withholds every copy
+        bool ok = *reinterpret_cast<const volatile uint32_t*>(reinterpret_cast<const uint8_t*>(prm.status) +
+                                                               kWsInjectOff) == 0u;
         for (int t = blockIdx.x; t < tiles && ok; t += gridDim.x) {
             int g, j;
             tile_of(prm, G, t, g, j);

@@ -1,4 +1,5 @@
-"""Failure detection without a GPU fault: the multi-row kernel's bounded waits.
+"""Failure detection without a GPU fault: the multi-row kernels' bounded waits
+(the verify kernel and the many-row GEMM).
 The test withholds the rotated input through the workspace's injection word
 (a flag that nothing sets then), so every wait for it runs out after its 2 s
 limit; the kernel winds down and the host reads EXL3_ERR_TIMEOUT from the
@@ -32,3 +33,21 @@ def test_withheld_input_times_out_and_reports(oracle_mod, k, n):
     ref = oracle_mod.gemm_sampled(inp.x, inp.packed, inp.scale, inp.su, inp.sv, k, n, bits, blocks)
     yv = y.cpu().numpy().astype(np.float64)
     check_close(np.concatenate([yv[:, 128 * b:128 * (b + 1)] for b in blocks], axis=1), ref, "after timeout")
+
+
+def test_many_row_withheld_operands_time_out_and_report(oracle_mod):
+    import torch
+    from gemm_exl3_gemv_b200 import exl3 as ex
+    m, k, n, bits = 160, 256, 384, 3
+    spec = synth.MatrixSpec("tl", k, n, bits, m, seed=73)
+    inp = synth.make_inputs(spec)
+    args = [to_dev(a) for a in (inp.x, inp.packed, inp.scale, inp.su, inp.sv)]
+    ws = torch.zeros(int(ex.lib.exl3_large_m_workspace_bytes(m, k, n, bits)), dtype=torch.uint8, device="cuda")
+    ws[4:8] = 1                                   # inject: the GEMM's producer issues no copy
+    ex.gemm_large(*args, bits, fp32=True, workspace=ws)
+    assert ex.workspace_status(ws) == ex.EXL3_ERR_TIMEOUT
+    ws[4:8] = 0
+    y = ex.gemm_large(*args, bits, fp32=True, workspace=ws)
+    assert ex.workspace_status(ws) == ex.EXL3_OK
+    ref = oracle_mod.gemm(inp.x, inp.packed, inp.scale, inp.su, inp.sv, k, n, bits)
+    check_close(y.cpu().numpy().astype(np.float64), ref, "many rows after timeout")
