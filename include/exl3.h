@@ -102,10 +102,11 @@ EXL3_API int exl3_kernel_launches(int m, int k_in, int n_out, int bits);
  * exl3_workspace_status -- synchronises `stream`, then reads and clears the
  * workspace status word.  Returns EXL3_OK, or EXL3_ERR_TIMEOUT if a kernel
  * that used this workspace gave up a bounded wait (its output is then not
- * valid).  Every wait in the multi-row kernel gives up after 2 s.
+ * valid).  Every wait in the multi-row kernels gives up after 2 s.
  * Testing that path: while the uint32 at byte offset 4 of the workspace is
- * nonzero, exl3_gemm_small_m (m >= 2) withholds the rotated input from its
- * product kernel, so every wait for it runs out; the call then finishes with
+ * nonzero, exl3_gemm_small_m (m >= 2), exl3_gemm_siblings (m >= 2) and
+ * exl3_gemm_large_m withhold the operand copies from their product kernels,
+ * so every wait for them runs out; the call then finishes with
  * EXL3_ERR_TIMEOUT here.  Keep that word zero in normal use.
  */
 EXL3_API int exl3_workspace_status(void *workspace, void *stream);
