@@ -1,8 +1,11 @@
-// exl3_aop.cuh -- the tensor-core A operand of the trellis products: one
-// tile row of a 128-channel output block (128 channels x 16 input rows, fp16,
-// MN-major, 128-byte swizzle: 4 KB), written by the lanes of one warp straight
-// from their decoded weights.  Used by the verify kernel (into shared memory)
-// and by the large-M path (into a global image of the whole matrix).
+// exl3_aop.cuh -- the tensor-core operands of the trellis products.
+//   A: one tile row of a 128-channel output block (128 channels x 16 input
+//      rows, fp16, MN-major, 128-byte swizzle: 4 KB), written by the lanes of
+//      one warp straight from their decoded weights.  Used by the verify
+//      kernel (into shared memory) and by the large-M path (into a global
+//      image of the whole matrix).
+//   B: the rotated input H(su .* x) in the matching K order (xt_rotate_item),
+//      used by the large-M path's pre-pass.
 #pragma once
 #include <cstdint>
 #include <utility>
