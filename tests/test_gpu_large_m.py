@@ -45,6 +45,24 @@ def test_model_shapes_sampled(ex, oracle_mod, m, n):
     check_close(got, ref, f"m={m} n={n}")
 
 
+@pytest.mark.parametrize("m,k,n,bits", [
+    (1100, 256, 17408, 3),      # 680 tiles of 256 rows on 148 persistent CTAs; row-tile-fastest order
+    (8192, 256, 1024, 2),       # 256 tiles; output-block-fastest order
+])
+def test_persistent_multi_tile_sampled(ex, oracle_mod, m, k, n, bits):
+    """Several tiles per persistent CTA: both tensor-memory accumulators in
+    turn, the ring running on across tiles, and each tile order."""
+    spec = synth.MatrixSpec("lgp", k, n, bits, m, seed=85)
+    inp = synth.make_inputs(spec)
+    G = n // 128
+    blocks = sorted({0, 1, G // 2, G - 1})
+    rows = sorted({0, 255, 256, m // 2, m - 257, m - 1})
+    ref = oracle_mod.gemm_sampled(inp.x[rows], inp.packed, inp.scale, inp.su, inp.sv, k, n, bits, blocks)
+    y = ex.gemm_large(*_args(inp, m), bits, fp32=True).cpu().numpy().astype(np.float64)[rows]
+    got = np.concatenate([y[:, 128 * b:128 * (b + 1)] for b in blocks], axis=1)
+    check_close(got, ref, f"m={m} k={k} n={n}")
+
+
 def test_agrees_with_verify_path_at_32_rows(ex):
     spec = synth.MatrixSpec("lgv", 5120, 1024, 4, 32, seed=83)
     inp = synth.make_inputs(spec)
