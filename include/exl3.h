@@ -215,8 +215,8 @@ EXL3_API int exl3_gemm_siblings(int m, const uint16_t *x, const uint16_t *su, co
                                 void *stream);
 
 /*
- * exl3_gemv_noalloc -- exl3_gemv without a workspace argument.  The paper has
- * no counterpart of this entry point; it exists for callers that cannot
+ * exl3_gemv_noalloc -- exl3_gemv without a workspace argument.  The source
+ * pages describe no counterpart of this entry point; it exists for callers that cannot
  * allocate device memory on the call path -- for example an inference engine
  * that reserves all of HBM for its own pool at start-up and forbids further
  * cudaMalloc, or a plugin whose host application owns the CUDA allocator --
