@@ -145,3 +145,19 @@ def test_large_m_validation(ex):
     assert f(*args(wsb=need - 1)) == ex.EXL3_ERR_WORKSPACE
     assert f(*args(ws=0)) == ex.EXL3_ERR_WORKSPACE
     assert f(*args(ws=16)) == ex.EXL3_ERR_MISALIGNED
+
+
+def test_large_m_workspace_layout(ex):
+    """Header (256 bytes), the decoded image (2 bytes per weight) and the rotated
+    input for m rows padded to the row tile: 256 rows when that gives 148 tiles,
+    else 128, else 64."""
+    def tile(m, n):
+        g = n // 128
+        for nb in (256, 128):
+            if g * ((m + nb - 1) // nb) >= 148:
+                return nb
+        return 64
+    for m, k, n in [(1, 128, 128), (300, 256, 256), (2048, 5120, 17408), (512, 5120, 5120), (8192, 5120, 5120)]:
+        nb = tile(m, n)
+        m_pad = (m + nb - 1) // nb * nb
+        assert ex.lib.exl3_large_m_workspace_bytes(m, k, n, 3) == 256 + k * n * 2 + m_pad * k * 2, (m, k, n)
