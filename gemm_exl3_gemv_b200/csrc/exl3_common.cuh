@@ -12,9 +12,10 @@ namespace exl3 {
 // ------------------------------------------------------------ workspace ---
 // [0, 256)            status word (uint32 at 0): nonzero after a timed-out wait;
 //                     word 1 (uint32 at 4): timeout injection for tests -- while
-//                     it is nonzero the verify kernel issues no copies of the
-//                     rotated input, so every wait for one runs out (zero in
-//                     normal use: the workspace is zero-filled)
+//                     it is nonzero (value v) each verify-kernel CTA issues only
+//                     its first v - 1 copies of the rotated input, so the wait
+//                     for the next one runs out (zero in normal use: the
+//                     workspace is zero-filled)
 // [256, 256 + 4*G)    one arrival counter per 128-channel output block
 // [ws_part_off, ...)  split-K partial sums, fp32 [splits][m][n_out]
 constexpr size_t kWsHeader = 256;

@@ -1,8 +1,8 @@
 // exl3_decode.cuh -- device-side trellis decoding for the EXL3 format.
 //
-// The pages name the EXL3 trellis format ("~3.2 bits/weight in the EXL3
-// trellis format", orcasaq2-rocm README, opening paragraph; "EXL3, 3.0 bpw",
-// exl3-rdna4-recipe, opening paragraph) without defining it.  The definition
+// The pages name the EXL3 trellis format (models at about 3 bits per weight:
+// orcasaq2-rocm README and exl3-rdna4-recipe, opening paragraphs) without
+// defining it.  The definition
 // used here is the specification's: 16x16 tiles, each a tail-biting stream of
 // 256*K bits; weight i of a tile is decoded from the 16-bit window that ends
 // at stream bit (i+1)*K, through the 3INST map.  Readings where the

@@ -2,8 +2,8 @@
 // whole matrix once into the tensor-core operand layout, then a tcgen05 GEMM.
 //
 // What is computed (the prompt-processing side of the decode speeds on the
-// orcasaq2-rocm README -- "Prefill: 1100-1800 tok/s at 8-32k", paragraph below
-// its speed table -- and of the exl3-rdna4-recipe page, "What you get"):
+// orcasaq2-rocm README -- the prefill rates given below its speed table -- and
+// of the exl3-rdna4-recipe page, "What you get"):
 //     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: m x K_in, y: m x N_out
 // At large m each decoded weight feeds 2m flops, so the decode is paid once per
 // call and the contraction runs as a dense tensor-core GEMM:

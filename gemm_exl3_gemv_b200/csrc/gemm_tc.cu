@@ -1,9 +1,9 @@
 // gemm_tc.cu -- the verify-batch product (2..32 input rows) on the 5th-generation
 // tensor cores (tcgen05), with the trellis decode on the CUDA cores.
 //
-// What is computed (the "WMMA GEMV for draft verification" and "batched
-// verification up to 32 rows" of the exl3-rdna4-recipe page, section "What we
-// added on top of upstream", here on B200):
+// What is computed (the exl3-rdna4-recipe page verifies drafted tokens with a
+// tensor-core GEMV and keeps verify batches of up to 32 rows on its fast
+// kernel, section "What we added on top of upstream"; here on B200):
 //     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: m x K_in, y: m x N_out
 //
 // Design:
@@ -77,8 +77,8 @@ struct TcLayout {
     static constexpr int off_z = off_a;                       // z [NT][128] fp32, over the A stages (segment end)
     static constexpr int off_b = off_a + kDec * kAStages * kABytes;
     static constexpr int off_bar = off_b + kBStages * BUNIT;
-    // aempty[kDec][kAStages], bfull[kBStages], bempty[kBStages], segdone
-    static constexpr int nbar = kDec * kAStages + 2 * kBStages + 1;
+    // aempty[kDec][kAStages], bfull[kBStages], bempty[kBStages], segdone, lastbar
+    static constexpr int nbar = kDec * kAStages + 2 * kBStages + 2;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;       // + slack to align the base to 1024
     static_assert(off_b % 1024 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     uint64_t* bfull = aempty + kDec * kAStages;               // [kBStages]: xt unit landed
     uint64_t* bempty = bfull + kBStages;                      // [kBStages]: all 8 MMAs on it completed
     uint64_t* segdone = bempty + kBStages;                    // every accumulator final
+    uint64_t* lastbar = segdone + 1;                          // every MMA of the CTA completed
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
     volatile int* abort_flag = misc + 1;
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
@@ -249,6 +250,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         for (int i = 0; i < kDec * kAStages; ++i) mbar_init(&aempty[i], 1);
         for (int i = 0; i < kBStages; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kDec); }
         mbar_init(segdone, kDec);
+        mbar_init(lastbar, kDec);
         misc[1] = 0;
         misc[2] = 0;
         fence_mbar_init();
@@ -267,25 +269,26 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         grid_dep_wait();               // xt is written by the pre-pass
         // ------------------------------------------------- xt producer ---
         // xt of unit (g, c) is chunks 2c, 2c+1: BUNIT contiguous bytes.
-        // a nonzero injection word (tests of the timeout path) leaves every
-        // decoder's wait for its xt unit to run out
-        const bool inject = *reinterpret_cast<const volatile uint32_t*>(a.ws + kWsInjectOff) != 0u;
-        if (lane == 0 && !inject) {
+        // A nonzero injection word v (tests of the timeout path) lets only the
+        // CTA's first v - 1 xt copies through, so the decoders' wait for the
+        // next one runs out (with MMAs of the earlier units possibly in flight).
+        const uint32_t inject = *reinterpret_cast<const volatile uint32_t*>(a.ws + kWsInjectOff);
+        const long long allowed = inject ? (long long)inject - 1 : (b1 - b0);
+        if (lane == 0) {
             int kk = 0;
             int c = (int)(b0 % C);
-            for (long long u = b0; u < b1; ++u, ++kk) {
+            for (long long u = b0; u < b1 && kk < allowed; ++u, ++kk) {
                 const int s = kk & (kBStages - 1);
                 if (kk >= kBStages && !wait_or_abort(&bempty[s], (uint32_t)(kk / kBStages - 1) & 1u, abort_flag)) break;
                 mbar_arrive_expect_tx(&bfull[s], L::BUNIT);
                 bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
                 if (++c == C) c = 0;
             }
-            // on abort, let every issued copy land before the CTA can exit
+            // every issued copy lands before the CTA can exit (a no-op wait in
+            // a normal run: the decoders have consumed them)
             const int issued = kk;
-            for (int v = issued > kBStages ? issued - kBStages : 0; v < issued; ++v) {
-                if (*abort_flag)
-                    (void)mbar_wait_bounded(&bfull[v & (kBStages - 1)], (uint32_t)(v / kBStages) & 1u, 100000000ull);
-            }
+            for (int v = issued > kBStages ? issued - kBStages : 0; v < issued; ++v)
+                (void)mbar_wait_bounded(&bfull[v & (kBStages - 1)], (uint32_t)(v / kBStages) & 1u, 100000000ull);
         }
     } else {
         // --------------------------------------------- decoder warps ---
@@ -368,9 +371,9 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             }
             if (k < nseg) unit(wa, k, kk + k);
             kk += nseg;
-            ok = __shfl_sync(0xffffffffu, (ok && !fail0) ? 1 : 0, 0) != 0;
-            if (ok) mma_commit_elect(segdone);           // arrives once this warp's MMAs are done
-            else if (lane == 0) mbar_arrive(segdone);
+            // arrives once every MMA this warp issued has completed -- also after a
+            // wait gave up part-way (then it covers the MMAs already in flight)
+            mma_commit_elect(segdone);
 
             // ---- accumulators -> zsm[NT][128] (the eight summed in a fixed order) ----
             int okd = 1;
@@ -431,6 +434,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             tc_fence_after();
             u0 = u1;
         }
+        mma_commit_elect(lastbar);                           // arrives once this warp's last MMA completed
     }
 
     // ---- cluster mode: the cluster's CTAs add their z in rank order
@@ -466,6 +470,10 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     }
 
     // ------------------------------------------------------------ teardown ---
+    // Every issued MMA completes (its operands are in shared memory already),
+    // so this wait ends even after an aborted run; only then may the tensor
+    // memory and the barriers its commits arrive on go away.
+    if (threadIdx.x == 0) (void)mbar_wait_bounded(lastbar, 0u, 100000000ull);
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {

@@ -1,8 +1,8 @@
 // gemv_m1.cu -- the single-row product (the decode-time GEMV) on CUDA cores.
 //
 // What is computed (the matrix-vector step behind the decode speeds of the
-// orcasaq2-rocm README, "EXL3 GEMM kernels were rewritten for RDNA's vector
-// ALUs", second paragraph):
+// orcasaq2-rocm README, whose second paragraph moves the EXL3 products onto
+// the GPU's vector ALUs):
 //     y = sv .* H( scale .* ( H(su .* x) W ) ),   x: 1 x K_in,  y: 1 x N_out
 // with W decoded on the fly from the trellis stream (exl3_decode.cuh).
 //

@@ -3,12 +3,12 @@
  * against EXL3-style trellis-quantised weights on NVIDIA B200 (sm_100a).
  *
  * What is computed.  The pages this library follows name the EXL3 trellis
- * format and its decode-time GEMV without defining it ("~3.2 bits/weight in
- * the EXL3 trellis format", orcasaq2-rocm README, opening paragraph; "EXL3
- * GEMM kernels were rewritten for RDNA's vector ALUs", same page, second
- * paragraph; "checking 8 drafted tokens", "batched verification up to 32
- * rows", exl3-rdna4-recipe, section "What we added on top of upstream").  The
- * format fixed here:
+ * format (a 27B-class model at a little over 3 bits per weight; orcasaq2-rocm
+ * README, opening paragraph) and its decode-time product, which that page's
+ * port moved onto the GPU's vector ALUs (same page, second paragraph), and a
+ * tensor-core GEMV that verifies a handful of drafted tokens, with verify
+ * batches of up to 32 rows (exl3-rdna4-recipe, section "What we added on top
+ * of upstream"), but they never define the format.  The format fixed here:
  *   - W is K_in x N_out, stored as 16x16 tiles; tile (tk, tn) is tile number
  *     tk*(N_out/16) + tn and holds 8*K uint32 words (K = bits per weight) that
  *     form one tail-biting bitstream of 256*K bits.  Stream bit j is bit
@@ -104,10 +104,11 @@ EXL3_API int exl3_kernel_launches(int m, int k_in, int n_out, int bits);
  * that used this workspace gave up a bounded wait (its output is then not
  * valid).  Every wait in the multi-row kernels gives up after 2 s.
  * Testing that path: while the uint32 at byte offset 4 of the workspace is
- * nonzero, exl3_gemm_small_m (m >= 2), exl3_gemm_siblings (m >= 2) and
- * exl3_gemm_large_m withhold the operand copies from their product kernels,
- * so every wait for them runs out; the call then finishes with
- * EXL3_ERR_TIMEOUT here.  Keep that word zero in normal use.
+ * nonzero, exl3_gemm_small_m (m >= 2) and exl3_gemm_siblings (m >= 2) let
+ * only the first v - 1 rotated-input copies of each CTA through (v = the
+ * word's value; v = 1 withholds them all), and exl3_gemm_large_m withholds
+ * every operand copy; the waits for the withheld copies run out and the call
+ * finishes with EXL3_ERR_TIMEOUT here.  Keep that word zero in normal use.
  */
 EXL3_API int exl3_workspace_status(void *workspace, void *stream);
 
@@ -188,10 +189,11 @@ EXL3_API int exl3_gemm_large_m(int m, const uint16_t *x, const uint32_t *packed,
  * exl3_gemm_siblings -- the product for a group of matrices that take the
  * same input: y_i = sv_i .* H(scale_i .* (H(su .* x) W_i)) for i < n_mats,
  * in one pass that rotates x once and spreads all the groups' output blocks
- * over the GPU together.  This is the sibling fusion the exl3-rdna4-recipe
- * page describes for verify batches ("a fused C++ MLP path", section "What we
- * added on top of upstream"): gate and up of an MLP, or q, k and v of an
- * attention block, whose inputs are the same activation rows.
+ * over the GPU together.  The exl3-rdna4-recipe page fuses the MLP's
+ * matrices into one native-code path for its verify batches (section "What
+ * we added on top of upstream"); this is that fusion here: gate and up of an
+ * MLP, or q, k and v of an attention block, whose inputs are the same
+ * activation rows.
  *   x, su  : as exl3_gemm_small_m, shared by every matrix of the group.
  *   mats   : HOST array of n_mats (1..8) exl3_matrix_t; each gives its packed
  *            words, scale, sv and output y (m x n_out, row-major) and n_out

@@ -8,9 +8,9 @@
  *
  * What it computes, and where each step comes from:
  *
- *   The pages name the format ("~3.2 bits/weight in the EXL3 trellis format",
- *   orcasaq2-rocm README, opening paragraph; "EXL3, 3.0 bpw ... SC_3.00bpw_H4",
- *   exl3-rdna4-recipe, opening paragraph) but never define it.  The definition
+ *   The pages name the format (27B-class models at about 3 bits per weight:
+ *   orcasaq2-rocm README and exl3-rdna4-recipe, opening paragraphs) but never
+ *   define it.  The definition
  *   written out below is the format specification this library follows:
  *   16x16 tiles, each a
  *   tail-biting bitstream of 256*K bits; weight i of a tile is decoded from the

@@ -14,8 +14,14 @@ from gpu_helpers import check_close, to_dev
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("k,n", [(640, 256), (256, 65536)])     # cluster cut; stream-K cut
-def test_withheld_input_times_out_and_reports(oracle_mod, k, n):
+# (k, n, v): v = 1 withholds every rotated-input copy; v = 3 lets each CTA's
+# first two through, so the CTAs with more units have MMAs issued (possibly
+# still in flight) when their wait for the third runs out
+@pytest.mark.parametrize("k,n,v", [(640, 256, 1),        # cluster cut, nothing issued
+                                   (256, 65536, 1),      # stream-K cut, nothing issued
+                                   (5120, 256, 3),       # cluster cut, 4 units per CTA
+                                   (256, 65536, 3)])     # stream-K cut, 3-4 units per CTA
+def test_withheld_input_times_out_and_reports(oracle_mod, k, n, v):
     import torch
     from gemm_exl3_gemv_b200 import exl3 as ex
     m, bits = 8, 3
@@ -23,7 +29,7 @@ def test_withheld_input_times_out_and_reports(oracle_mod, k, n):
     inp = synth.make_inputs(spec)
     args = [to_dev(a) for a in (inp.x, inp.packed, inp.scale, inp.su, inp.sv)]
     ws = ex.alloc_workspace(m, k, n, bits)
-    ws[4:8] = 1                                   # inject: withhold the rotated input
+    ws[4:8] = torch.tensor([v, 0, 0, 0], dtype=torch.uint8)   # inject: withhold the rotated input
     ex.gemm(*args, bits, fp32=True, workspace=ws)
     assert ex.workspace_status(ws) == ex.EXL3_ERR_TIMEOUT
     ws[4:8] = 0
