@@ -5,8 +5,11 @@ One step = one pass of every matrix product of the stack (64 layers x
 {q, k, v, o, gate, up, down}, bits per layer drawn from seed 4) at M = 32 rows
 (the draft-verification batch), each product running the whole hot path:
 input rotation, packed-stream load, trellis decode, contraction, split-K
-reduction, scale and output rotation.  The same stack at M = 1 (decode) is
-timed too and reported as us/layer.
+reduction, scale and output rotation.  Each layer's seven products are one
+grouped library call (one rotation pre-pass and one product launch), unless
+--separate.  The same stack at M = 1 (decode), 8 and 16 is timed too and
+reported as us/layer, and so is the chained stack (each layer's output is the
+next layer's input, one CUDA graph) at M = 32 and M = 1.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -47,12 +50,15 @@ def parse():
                     help="input rows; above 32 the products go through the many-row (prefill) call, "
                          "with the synthetic rows repeated to m")
     ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--separate", action="store_true", help="one library call per matrix instead of per layer")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="time only the main row count (no M=1/8/16, no chain)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ref-budget", type=float, default=None,
                     help="seconds of oracle work per step for --impl reference (default: about 90 s per run)")
     ap.add_argument("--only", default=None,
                     help="restrict the stack to one matrix kind (q,k,v,o,gate,up,down), e.g. for ncu captures")
+    ap.add_argument("--oracle-sample", nargs=2, type=float, default=None, help=argparse.SUPPRESS)
     return ap.parse_args()
 
 
@@ -63,32 +69,24 @@ def dist_env():
     return world, rank, local
 
 
-KERNEL_SOURCES = ["gemm_exl3_gemv_b200/csrc/gemm_tc.cu", "gemm_exl3_gemv_b200/csrc/exl3_aop.cuh",
-                  "gemm_exl3_gemv_b200/csrc/exl3_decode.cuh",
-                  "gemm_exl3_gemv_b200/csrc/exl3_common.cuh", "gemm_exl3_gemv_b200/csrc/exl3_tc.cuh"]
+# ------------------------------------------------- committed ncu counters ----
 
-
-def kernel_source_hash():
+def counters(name):
+    """A committed ncu counter record (profiles/<name>.json) -- only if the
+    kernel sources it was measured on are unchanged (else None, reason)."""
     import hashlib
-    h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
-    return h.hexdigest()
-
-
-def measured_traffic_ratio():
-    """DRAM bytes per packed-weight byte of the verify-GEMM kernel, from the
-    committed ncu capture in profiles/ -- only if the kernel's sources are the
-    ones that capture measured (else None)."""
-    p = os.path.join(ROOT, "profiles", "gemm_tc_traffic.json")
+    p = os.path.join(ROOT, "profiles", name + ".json")
     if not os.path.exists(p):
-        return None, None
+        return None, "no committed capture"
     with open(p) as f:
         d = json.load(f)
-    if d.get("source_sha256") != kernel_source_hash():
-        return None, None
-    return float(d["dram_bytes_per_packed_byte"]), d.get("capture")
+    h = hashlib.sha256()
+    for rel in d.get("sources", []):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    if d.get("source_sha256") != h.hexdigest():
+        return None, "kernel sources changed since the capture"
+    return d, None
 
 
 def load_peaks():
@@ -174,19 +172,29 @@ def cores_used():
         return os.cpu_count() or 1
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 _INPUT_CACHE = {}
 
 
 def oracle_sample(budget_s: float, m: int):
     """Time the fp64 oracle on layer-0 matrices (smallest first: k, v, q, o,
     gate, up, down) until `budget_s` is spent; returns (packed bytes, seconds,
-    names).  Input generation is outside the timed region."""
+    [(name, us)]).  Input generation is outside the timed region."""
     import oracle
     oracle.build()
     specs = [s for s in synth.workload(5, m=m) if s.layer == 0]
-    # smallest first so that a short budget still covers at least one matrix
     specs = sorted(specs, key=lambda s: s.n_weights)
-    done_b, done_t, names = 0, 0.0, []
+    done_b, done_t, per = 0, 0.0, []
     for spec in specs:
         if spec not in _INPUT_CACHE:
             _INPUT_CACHE[spec] = synth.make_inputs(spec)
@@ -196,10 +204,41 @@ def oracle_sample(budget_s: float, m: int):
         dt = time.perf_counter() - t0
         done_b += spec.packed_bytes
         done_t += dt
-        names.append(spec.name)
+        per.append((spec.name, round(dt * 1e6, 1)))
         if done_t >= budget_s:
             break
-    return done_b, done_t, names
+    return done_b, done_t, per
+
+
+def oracle_sample_threads(budget_s: float, m: int, threads: int):
+    """oracle_sample in a fresh process limited to `threads` OpenMP threads."""
+    env = dict(os.environ, OMP_NUM_THREADS=str(threads))
+    out = subprocess.run([sys.executable, os.path.abspath(__file__), "--oracle-sample", str(budget_s), str(m)],
+                         env=env, capture_output=True, text=True, timeout=600)
+    if out.returncode != 0:
+        return None
+    return json.loads(out.stdout.strip().splitlines()[-1])
+
+
+def cpu_baseline(m: int, budget_s: float, single_budget_s: float):
+    """The fp64 oracle as it stands, on this host's cores (all, and one)."""
+    cores = cores_used()
+    allc = oracle_sample_threads(budget_s, m, cores)
+    one = oracle_sample_threads(single_budget_s, m, 1)
+    if allc is None:
+        return None
+    layer_bytes = sum(s.packed_bytes for s in synth.workload(5, m=m) if s.layer == 0)
+    gbs = allc["bytes"] / allc["seconds"] / 1e9
+    d = {"value": round(gbs, 6), "unit": UNIT, "cores": cores, "kind": "oracle",
+         "sample": f"fp64 oracle (C, OpenMP) on layer-0 matrices {','.join(n for n, _ in allc['per'])} at M={m}",
+         "cpu_model": cpu_model(),
+         "us_per_matrix": dict(allc["per"]),
+         "us_per_layer_est": round(layer_bytes / (gbs * 1e9) * 1e6, 1)}
+    if one is not None:
+        g1 = one["bytes"] / one["seconds"] / 1e9
+        d["single_thread"] = {"value": round(g1, 6), "unit": UNIT, "us_per_matrix": dict(one["per"]),
+                              "us_per_layer_est": round(layer_bytes / (g1 * 1e9) * 1e6, 1)}
+    return d
 
 
 def run_reference(args, world, rank):
@@ -211,10 +250,10 @@ def run_reference(args, world, rank):
     per_step_budget = args.ref_budget if args.ref_budget is not None else max(1.0, 90.0 / max(1, steps + warmup))
     vals, samples = [], None
     for i in range(warmup + steps):
-        b, t, names = oracle_sample(per_step_budget, args.m)
+        b, t, per = oracle_sample(per_step_budget, args.m)
         if i >= warmup:
             vals.append(b / t / 1e9)
-        samples = names
+        samples = [n for n, _ in per]
     value = statistics.median(vals)
     sample = f"fp64 oracle on layer-0 matrices {','.join(samples)} at M={args.m}, per step"
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT,
@@ -222,7 +261,7 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "m": args.m, "layers": args.layers},
             "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cores_used(),
-                             "kind": "oracle", "sample": sample},
+                             "kind": "oracle", "sample": sample, "cpu_model": cpu_model()},
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -235,99 +274,6 @@ def make_weights(torch, device, layers, only=None):
     if only:
         specs = [s for s in specs if s.name.split(".")[1] == only]
     return specs, [synth.splitmix64_words_torch(s.stream_id, s.n_words, device) for s in specs]
-
-
-class Stack:
-    """The stack's products.  Inputs x and outputs y of all matrices live in one
-    flat device buffer each (and one pinned host buffer each), with a layer's
-    matrices contiguous, so that the end-to-end step moves one slice per layer."""
-
-    def __init__(self, ex, torch, device, m, specs, weights):
-        self.specs = specs
-        self.m = m
-        self.mats = []
-        ws_need = 0
-        x_off, y_off, xo, yo = [], [], 0, 0
-        for spec in specs:
-            x_off.append(xo)
-            y_off.append(yo)
-            xo += m * spec.k_in
-            yo += m * spec.n_out
-        self.x_dev = torch.empty(xo, dtype=torch.float16, device=device)
-        self.y_dev = torch.empty(yo, dtype=torch.float16, device=device)
-        self.x_pin = torch.empty(xo, dtype=torch.float16).pin_memory()
-        self.y_pin = torch.empty(yo, dtype=torch.float16).pin_memory()
-        self.large = m > 32
-        for i, (spec, packed) in enumerate(zip(specs, weights)):
-            scale, x, su, sv = synth.small_inputs(spec)
-            if x.shape[0] < m:                          # many-row runs: the synthetic rows repeated
-                x = np.tile(x, ((m + x.shape[0] - 1) // x.shape[0], 1))
-            t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-            xs = slice(x_off[i], x_off[i] + m * spec.k_in)
-            ys = slice(y_off[i], y_off[i] + m * spec.n_out)
-            self.x_pin[xs].copy_(torch.from_numpy(np.ascontiguousarray(x[:m]).reshape(-1)))
-            self.x_dev[xs].copy_(self.x_pin[xs])
-            self.mats.append({"spec": spec, "packed": packed, "scale": t(scale), "su": t(su), "sv": t(sv),
-                              "x": self.x_dev[xs].view(m, spec.k_in), "y": self.y_dev[ys].view(m, spec.n_out)})
-            ws_need = max(ws_need, int(ex.lib.exl3_large_m_workspace_bytes(m, spec.k_in, spec.n_out, spec.bits))
-                          if self.large else ex.workspace_bytes(m, spec.k_in, spec.n_out, spec.bits))
-        # per layer: its matrices and its contiguous x and y slices
-        self.layers = []
-        for i, spec in enumerate(specs):
-            if not self.layers or self.layers[-1]["layer"] != spec.layer:
-                self.layers.append({"layer": spec.layer, "mats": [], "x0": x_off[i], "y0": y_off[i]})
-            lay = self.layers[-1]
-            lay["mats"].append(self.mats[i])
-            lay["x1"] = x_off[i] + m * spec.k_in
-            lay["y1"] = y_off[i] + m * spec.n_out
-        self.s_in = torch.cuda.Stream(device=device)
-        self.s_out = torch.cuda.Stream(device=device)
-        self.ws = torch.zeros(ws_need, dtype=torch.uint8, device=device)
-        self.ex = ex
-        self.packed_bytes = sum(s.packed_bytes for s in self.specs)
-        # the many-row call launches three kernels (decode image, input rotation, GEMM)
-        self.launches = sum(3 if self.large else ex.kernel_launches(m, s.k_in, s.n_out, s.bits)
-                            for s in self.specs)
-        self.io_bytes = sum(2 * m * (s.k_in + s.n_out) + 2 * (s.k_in + 2 * s.n_out) for s in self.specs)
-        self.h2d = self.x_pin.numel() * 2
-        self.d2h = self.y_pin.numel() * 2
-
-    def run_mats(self, mats):
-        ex = self.ex
-        call = ex.gemm_large if self.large else ex.gemm
-        for mt in mats:
-            call(mt["x"], mt["packed"], mt["scale"], mt["su"], mt["sv"], mt["spec"].bits, out=mt["y"],
-                 workspace=self.ws)
-
-    def run(self):
-        self.run_mats(self.mats)
-
-    def run_e2e(self, torch):
-        """One end-to-end step from pinned host buffers: per layer, its inputs go
-        up on one stream, its products run on the current stream, its outputs come
-        down on a third, so the copies of one layer overlap the products of its
-        neighbours.  Every copy is inside the step; the step ends when the last
-        output has landed on the host."""
-        cs = torch.cuda.current_stream()
-        start = torch.cuda.Event()
-        start.record(cs)
-        self.s_in.wait_event(start)
-        self.s_out.wait_event(start)
-        for lay in self.layers:
-            xs, ys = slice(lay["x0"], lay["x1"]), slice(lay["y0"], lay["y1"])
-            with torch.cuda.stream(self.s_in):
-                self.x_dev[xs].copy_(self.x_pin[xs], non_blocking=True)
-                ev_in = torch.cuda.Event()
-                ev_in.record(self.s_in)
-            cs.wait_event(ev_in)
-            self.run_mats(lay["mats"])
-            ev_out = torch.cuda.Event()
-            ev_out.record(cs)
-            self.s_out.wait_event(ev_out)
-            with torch.cuda.stream(self.s_out):
-                self.y_pin[ys].copy_(self.y_dev[ys], non_blocking=True)
-        cs.wait_stream(self.s_in)
-        cs.wait_stream(self.s_out)
 
 
 def timed(torch, fn, steps, warmup, barrier):
@@ -357,6 +303,7 @@ def run_ours(args, world, rank, local):
     barrier = (lambda: dist.barrier()) if dist else (lambda: None)
 
     from gemm_exl3_gemv_b200 import exl3 as ex
+    from gemm_exl3_gemv_b200.stack import Stack
 
     def max_over_ranks(v):
         if not dist:
@@ -365,66 +312,86 @@ def run_ours(args, world, rank, local):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    results = {}
-    graphs = []
     specs, weights = make_weights(torch, device, args.layers, args.only)
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
-    for m in ([args.m, 1] if args.m != 1 else [1]):
-        st = Stack(ex, torch, device, m, specs, weights)
-        st.run()                                        # first call configures kernels
+    full_layers = args.only is None
+    extra = not args.no_extra and args.m <= 32
+    rows = [args.m]
+    if extra:
+        rows += [m for m in (1, 16, 8) if m != args.m]
+
+    def graph_or_eager(st, fn):
+        fn()                                            # the configuring first call, outside any capture
         torch.cuda.synchronize()
-        fn = st.run
-        launch = "eager"
-        if not args.no_graph:
-            try:
-                g = torch.cuda.CUDAGraph()
-                with torch.cuda.graph(g):
-                    st.run()
-                graphs.append(g)
-                fn = g.replay
-                launch = "cuda_graph"
-            except Exception as e:  # capture unsupported: time eager launches
-                print(f"# graph capture failed ({e}); timing eager launches", file=sys.stderr)
+        if args.no_graph:
+            return fn, None, "eager"
+        try:
+            g = st.capture(fn)
+            return g.replay, g, "cuda_graph"
+        except Exception as e:  # capture unsupported: time eager launches
+            print(f"# graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            return fn, None, "eager"
+
+    results = {}
+    main_stack = None
+    for m in rows:
+        st = Stack(ex, torch, device, m, specs, weights, mode="sweep", grouped=not args.separate)
+        fn, g, launch = graph_or_eager(st, st.run)
         sampler = ClockSampler(gpu_id) if m == args.m else None
         if sampler:
             sampler.start()
             time.sleep(0.5)                             # let nvidia-smi start sampling
-        ms = timed(torch, fn, args.steps, args.warmup, barrier)
+        ms = max_over_ranks(timed(torch, fn, args.steps, args.warmup, barrier))
         clocks = sampler.stop() if sampler else None
-        ms = max_over_ranks(ms)
-        res = {"stack": st, "ms": ms, "launch": launch, "clocks": clocks}
+        res = {"ms": ms, "launch": launch, "clocks": clocks, "launches": st.launches()}
         if m == args.m:
-            st.run_e2e(torch)
-            torch.cuda.synchronize()
-            fn_e2e = lambda: st.run_e2e(torch)
-            res["e2e_launch"] = "eager"
-            if not args.no_graph:
-                try:
-                    ge = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(ge):
-                        st.run_e2e(torch)
-                    graphs.append(ge)
-                    fn_e2e = ge.replay
-                    res["e2e_launch"] = "cuda_graph"
-                except Exception as e:  # capture unsupported: time eager launches
-                    print(f"# e2e graph capture failed ({e}); timing eager launches", file=sys.stderr)
-            res["e2e_ms"] = max_over_ranks(timed(torch, fn_e2e, args.steps, max(1, args.warmup), barrier))
+            # end to end through the binding from pinned host buffers: graphed, then eager
+            fe, ge, elaunch = graph_or_eager(st, st.run_e2e)
+            res["e2e_ms"] = max_over_ranks(timed(torch, fe, args.steps, max(1, args.warmup), barrier))
+            res["e2e_launch"] = elaunch
+            res["e2e_eager_ms"] = max_over_ranks(timed(torch, st.run_e2e, args.steps, max(1, args.warmup), barrier))
             assert ex.workspace_status(st.ws) == ex.EXL3_OK
             assert torch.equal(st.y_pin, st.y_dev.cpu()), "end-to-end outputs differ from the device outputs"
+            del ge
+            main_stack = st
+        assert ex.workspace_status(st.ws) == ex.EXL3_OK
+        del g
         results[m] = res
         if m != args.m:
             del st
         torch.cuda.synchronize()
 
+    chain = {}
+    if extra and full_layers:
+        for m in ([args.m, 1] if args.m != 1 else [1]):
+            st = Stack(ex, torch, device, m, specs, weights, mode="chain")
+            fn, g, launch = graph_or_eager(st, st.run)
+            chain[m] = max_over_ranks(timed(torch, fn, args.steps, args.warmup, barrier))
+            assert ex.workspace_status(st.ws) == ex.EXL3_OK
+            del g, st
+
     main = results[args.m]
-    st = main["stack"]
-    layers = args.layers
+    st = main_stack
+    layers = len(st.layers)
     gbs = st.packed_bytes / (main["ms"] * 1e-3) / 1e9
     peak, peak_kind = load_peaks()
     algo_bytes = st.packed_bytes + st.io_bytes
     achieved = algo_bytes / (main["ms"] * 1e-3) / 1e9
-    ratio, traffic_src = measured_traffic_ratio() if 1 < args.m <= 32 else (None, None)
-    traffic = round(ratio * st.packed_bytes / len(st.specs)) if ratio else None
+    n_weights = sum(s.n_weights for s in st.specs)
+    kname = "gemv_m1_counters" if args.m == 1 else "gemm_tc_counters"
+    cnt, cnt_why = counters(kname) if args.m <= 32 else (None, "many-row path")
+    traffic = None
+    if cnt is not None and "dram_bytes_per_packed_byte" in cnt:
+        traffic = round(cnt["dram_bytes_per_packed_byte"] * st.packed_bytes / len(st.specs))
+    sm_mhz = (main["clocks"] or {}).get("sm_mhz") or 1965.0
+    issue = None
+    if cnt is not None and "thread_instructions_per_weight" in cnt:
+        ipw = float(cnt["thread_instructions_per_weight"])
+        wps = n_weights / (main["ms"] * 1e-3)
+        peak_ti = 4 * 148 * sm_mhz * 1e6 * 32                 # 4 issue slots x 148 SMs x clock x 32 lanes
+        issue = {"bound": "alu-issue", "instr_per_weight": ipw, "weights_per_s": round(wps / 1e12, 4),
+                 "achieved": round(ipw * wps / 1e12, 3), "peak": round(peak_ti / 1e12, 3), "unit": "T thread-instr/s",
+                 "frac": round(ipw * wps / peak_ti, 4), "sm_mhz": sm_mhz, "source": cnt.get("capture")}
     line = {
         "metric": METRIC, "value": round(gbs * world, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms"], 4),
@@ -434,26 +401,31 @@ def run_ours(args, world, rank, local):
                    "m": args.m, "layers": layers,
                    "packed_bytes_per_step": st.packed_bytes,
                    "l2": "inputs larger than L2: %.2f GB of packed weights per step" % (st.packed_bytes / 1e9),
+                   "calls": "one grouped call per layer" if st.grouped else "one call per matrix",
                    "launch": main["launch"], "parallelism": f"replicas x{world}"},
         "us_per_layer_m%d" % args.m: round(main["ms"] * 1e3 / layers, 3),
         "pct_of_8TBps": round(100 * gbs / 8000.0, 2),
         "pct_of_measured_hbm": round(100 * gbs / peak, 2),
-        "gpu_launches": st.launches * args.steps,
+        "gpu_launches": main["launches"] * args.steps,
         "e2e": {"value": round(world * st.packed_bytes / (main["e2e_ms"] * 1e-3) / 1e9, 3), "unit": UNIT,
                 "h2d_bytes_per_step": st.h2d, "d2h_bytes_per_step": st.d2h,
                 "ms_per_step": round(main["e2e_ms"], 4),
-                "pipeline": "per layer: H2D stream -> products -> D2H stream, overlapped; " + main["e2e_launch"]},
+                "pipeline": "per layer: H2D stream -> products -> D2H stream, overlapped; " + main["e2e_launch"],
+                "eager": {"value": round(world * st.packed_bytes / (main["e2e_eager_ms"] * 1e-3) / 1e9, 3),
+                          "ms_per_step": round(main["e2e_eager_ms"], 4),
+                          "launch": "eager: every library call through the binding and the C ABI each step"}},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic,
                      "peak_kind": peak_kind,
-                     "kernel": "verify product (input-rotation pre-pass + gemm_tc_kernel), per product: "
-                               "algorithmic bytes / (CUDA-event step time / products)",
+                     "kernel": ("verify product (rotation pre-pass + gemm_tc_kernel)" if args.m > 1 else
+                                "single-row product (gemv_m1_kernel)") +
+                               ": algorithmic bytes per step / CUDA-event step time",
                      "algorithmic_bytes_per_product": round(algo_bytes / len(st.specs)),
-                     "traffic_source": traffic_src,
-                     "launches_per_step": st.launches},
+                     "traffic_source": cnt.get("capture") if cnt else cnt_why,
+                     "launches_per_step": main["launches"],
+                     "issue": issue if issue else {"bound": "alu-issue", "frac": None, "why": cnt_why}},
     }
     if st.large:
-        # many rows: a dense contraction on the tensor cores (fp16 in, fp32 accumulate)
         flops = sum(2.0 * args.m * s.k_in * s.n_out for s in st.specs)
         tflops = flops / (main["ms"] * 1e-3) / 1e12
         tpeak, tkind = load_tensor_peak()
@@ -462,21 +434,24 @@ def run_ours(args, world, rank, local):
                             "frac": round(tflops / tpeak, 4), "traffic": None, "peak_kind": tkind,
                             "kernel": "many-row product (decode image + input rotation + tcgen05 GEMM), "
                                       "2 m k n flops per product / (CUDA-event step time / products)",
-                            "traffic_source": None, "launches_per_step": st.launches}
-    if 1 in results and args.m != 1:
-        r1 = results[1]
-        line["us_per_layer_m1"] = round(r1["ms"] * 1e3 / layers, 3)
-        line["gbs_m1"] = round(st.packed_bytes / (r1["ms"] * 1e-3) / 1e9, 3)
-        line["pct_of_measured_hbm_m1"] = round(100 * line["gbs_m1"] / peak, 2)
+                            "traffic_source": None, "launches_per_step": main["launches"]}
+    m1_ms = results[1]["ms"] if 1 in results else None
+    for m, r in results.items():
+        if m == args.m:
+            continue
+        line["us_per_layer_m%d" % m] = round(r["ms"] * 1e3 / layers, 3)
+        line["gbs_m%d" % m] = round(st.packed_bytes / (r["ms"] * 1e-3) / 1e9, 3)
+    if m1_ms:
+        line["pct_of_measured_hbm_m1"] = round(100 * line.get("gbs_m1", gbs) / peak, 2)
+        line["step_vs_m1"] = {("m%d" % m): round(r["ms"] / m1_ms, 3) for m, r in results.items() if m != 1}
+    for m, ms in chain.items():
+        line["us_per_layer_chain_m%d" % m] = round(ms * 1e3 / layers, 3)
     if main["clocks"]:
         line["clocks"] = main["clocks"]
-    del graphs
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        os.environ.setdefault("OMP_NUM_THREADS", str(cores_used()))
-        b, t, names = oracle_sample(15.0, args.m)
-        line["cpu_baseline"] = {"value": round(b / t / 1e9, 6), "unit": UNIT, "cores": cores_used(),
-                                "kind": "oracle",
-                                "sample": f"fp64 oracle, layer-0 matrices {','.join(names)} at M={args.m}"}
+        cb = cpu_baseline(args.m, 12.0, 6.0)
+        if cb:
+            line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:
@@ -486,6 +461,10 @@ def run_ours(args, world, rank, local):
 
 def main():
     args = parse()
+    if args.oracle_sample is not None:
+        b, t, per = oracle_sample(args.oracle_sample[0], int(args.oracle_sample[1]))
+        print(json.dumps({"bytes": b, "seconds": t, "per": per}))
+        return
     world, rank, local = dist_env()
     if args.impl == "reference":
         run_reference(args, world, rank)

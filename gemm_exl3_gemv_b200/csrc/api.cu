@@ -51,21 +51,19 @@ int validate_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16
     return EXL3_OK;
 }
 
-// Problem description of a single product (a group of one sibling).
+// Problem description of a single product (a group of one member).
 exl3::GemmArgs single_args(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale,
                            const uint16_t* su, const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out,
                            int bits, void* ws)
 {
     exl3::GemmArgs a = {};
-    a.x = x;
-    a.su = su;
     a.y_fp32 = y_fp32 ? 1 : 0;
     a.m = m;
-    a.k_in = k_in;
     a.bits = bits;
-    a.n_out = n_out;
-    a.nsib = 1;
-    a.sib[0] = exl3::Sibling{packed, scale, sv, y, n_out, 0};
+    a.nmem = 1;
+    a.shared_x = 1;
+    a.mem[0] = exl3::Member{x, su, packed, scale, sv, y, k_in, n_out, 0, 0, 0, 0};
+    exl3::finish_group(a);
     a.ws = static_cast<unsigned char*>(ws);
     a.pdl = 1;
     return a;
@@ -215,7 +213,7 @@ extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, 
 {
     if (!x || !su || !mats) return EXL3_ERR_INVALID_ARG;
     if (m <= 0 || k_in <= 0 || n_mats <= 0) return EXL3_ERR_INVALID_ARG;
-    if (n_mats > exl3::kMaxSiblings || m > 32 || !bits_ok(bits) || k_in % 128) return EXL3_ERR_UNSUPPORTED;
+    if (n_mats > exl3::kMaxMembers || m > 32 || !bits_ok(bits) || k_in % 128) return EXL3_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(su)) return EXL3_ERR_MISALIGNED;
     exl3::GemmArgs a = {};
     long long total = 0;
@@ -226,7 +224,7 @@ extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, 
         if (t.n_out % 128) return EXL3_ERR_UNSUPPORTED;
         if (!aligned16(t.packed) || !aligned16(t.scale) || !aligned16(t.sv) || !aligned16(t.y))
             return EXL3_ERR_MISALIGNED;
-        a.sib[i] = exl3::Sibling{t.packed, t.scale, t.sv, t.y, t.n_out, (int)(total / 128)};
+        a.mem[i] = exl3::Member{x, su, t.packed, t.scale, t.sv, t.y, k_in, t.n_out, 0, 0, 0, 0};
         total += t.n_out;
     }
     if (total > (1LL << 30)) return EXL3_ERR_UNSUPPORTED;
@@ -235,16 +233,78 @@ extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, 
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
     int st = check_arch();
     if (st != EXL3_OK) return st;
-    a.x = x;
-    a.su = su;
     a.y_fp32 = y_fp32 ? 1 : 0;
     a.m = m;
-    a.k_in = k_in;
     a.bits = bits;
-    a.n_out = n_total;
-    a.nsib = n_mats;
+    a.nmem = n_mats;
+    a.shared_x = 1;
+    exl3::finish_group(a);
     a.ws = static_cast<unsigned char*>(workspace);
     a.pdl = 1;
+    cudaError_t e = launch_product(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
+}
+
+// ---------------------------------------------------------------- grouped ---
+
+namespace {
+
+// Validate a grouped call's problem list and fill the group description
+// (everything but the workspace).  Host only, no CUDA call.
+int grouped_args(int m, const exl3_problem_t* probs, int n_probs, int y_fp32, int bits, exl3::GemmArgs& a,
+                 bool check_ptrs)
+{
+    if (!probs || m <= 0 || n_probs <= 0) return EXL3_ERR_INVALID_ARG;
+    if (n_probs > exl3::kMaxMembers || m > 32 || !bits_ok(bits)) return EXL3_ERR_UNSUPPORTED;
+    a = exl3::GemmArgs{};
+    long long total = 0;
+    for (int i = 0; i < n_probs; ++i) {
+        const exl3_problem_t& t = probs[i];
+        if (check_ptrs && (!t.x || !t.su || !t.packed || !t.scale || !t.sv || !t.y)) return EXL3_ERR_INVALID_ARG;
+        if (t.k_in <= 0 || t.n_out <= 0) return EXL3_ERR_INVALID_ARG;
+        if (t.k_in % 128 || t.n_out % 128) return EXL3_ERR_UNSUPPORTED;
+        if (check_ptrs && (!aligned16(t.x) || !aligned16(t.su) || !aligned16(t.packed) || !aligned16(t.scale) ||
+                           !aligned16(t.sv) || !aligned16(t.y)))
+            return EXL3_ERR_MISALIGNED;
+        a.mem[i] = exl3::Member{t.x, t.su, t.packed, t.scale, t.sv, t.y, t.k_in, t.n_out, 0, 0, 0, 0};
+        total += t.n_out;
+    }
+    if (total > (1LL << 30)) return EXL3_ERR_UNSUPPORTED;
+    a.y_fp32 = y_fp32 ? 1 : 0;
+    a.m = m;
+    a.bits = bits;
+    a.nmem = n_probs;
+    a.shared_x = 0;
+    exl3::finish_group(a);
+    a.pdl = 1;
+    return EXL3_OK;
+}
+
+size_t grouped_ws(const exl3::GemmArgs& a)
+{
+    return a.m == 1 ? exl3::m1_group_workspace_bytes(a) : exl3::tc_group_workspace_bytes(a);
+}
+
+}  // namespace
+
+extern "C" size_t exl3_grouped_workspace_bytes(int m, const exl3_problem_t* probs, int n_probs, int bits)
+{
+    exl3::GemmArgs a;
+    if (grouped_args(m, probs, n_probs, 0, bits, a, false) != EXL3_OK) return 0;
+    return grouped_ws(a);
+}
+
+extern "C" int exl3_gemm_grouped(int m, const exl3_problem_t* probs, int n_probs, int y_fp32, int bits,
+                                 void* workspace, size_t ws_bytes, void* stream)
+{
+    exl3::GemmArgs a;
+    int st = grouped_args(m, probs, n_probs, y_fp32, bits, a, true);
+    if (st != EXL3_OK) return st;
+    if (!workspace || ws_bytes < grouped_ws(a)) return EXL3_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
+    st = check_arch();
+    if (st != EXL3_OK) return st;
+    a.ws = static_cast<unsigned char*>(workspace);
     cudaError_t e = launch_product(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }

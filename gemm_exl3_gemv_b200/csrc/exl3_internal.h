@@ -12,53 +12,95 @@ cudaError_t launch_decode_tiles(const uint32_t* packed, int k_in, int n_out, int
 cudaError_t launch_hadamard128(const uint16_t* in, uint16_t* out, const uint16_t* signs, int rows, int n, int mode,
                                cudaStream_t stream);
 
-// One product of a sibling group: the matrices that share the input x (and
-// its sign vector su), e.g. the gate and up projections of an MLP, or q, k
-// and v.  Output blocks of the group are numbered consecutively: sibling i
-// owns blocks [g0, g0 + n_out / 128).
-constexpr int kMaxSiblings = 8;
-struct Sibling {
+// A launch covers a group of 1..kMaxMembers products.  Member i has its own
+// weights (packed, scale, sv), output y and shape; its input rows x and sign
+// vector su are either its own (a grouped call: independent problems, e.g.
+// the seven matrices of a layer in a verify sweep) or shared by every member
+// (a sibling group: the gate and up projections of an MLP, or q, k and v).
+// Output blocks (128 channels) and work units of the group are numbered
+// member after member: member i owns blocks [g0, g0 + n_out/128) and units
+// [u0, u0 + units of member i) of the launching kernel.
+constexpr int kMaxMembers = 8;
+struct Member {
+    const uint16_t* x;        // m x k_in fp16 input rows
+    const uint16_t* su;       // k_in fp16 +-1
     const uint32_t* packed;   // trellis words (k_in x n_out)
     const uint16_t* scale;    // n_out fp16
     const uint16_t* sv;       // n_out fp16 +-1
     void* y;                  // m x n_out, fp16 or fp32
-    int n_out;
-    int g0;                   // first output block of this sibling
+    int k_in, n_out;
+    int g0;                   // first output block of this member
+    int pad_;
+    long long u0;             // first work unit of this member (set by the launching path)
+    long long xt0;            // verify path: byte offset of this member's rotated input in the x~ region
 };
 
 // Problem description shared by the product kernels.
 struct GemmArgs {
-    const uint16_t* x;        // m x k_in fp16
-    const uint16_t* su;       // k_in fp16 +-1
     int y_fp32;
-    int m, k_in, bits;
-    int n_out;                // total output width of the group (sum over siblings)
-    int nsib;                 // 1 .. kMaxSiblings
-    Sibling sib[kMaxSiblings];
+    int m, bits;
+    int n_out;                // total output width of the group (sum over members)
+    int k_max;                // largest k_in of the group
+    int nmem;                 // 1 .. kMaxMembers
+    int same_k;               // every member has the same k_in
+    int shared_x;             // every member takes the same x and su (sibling group)
+    Member mem[kMaxMembers];
     unsigned char* ws;        // workspace base
     int pdl;                  // launch with programmatic dependent launch (overlap the previous kernel's tail)
 };
 
+// Fill the group numbering (g0) and n_out / k_max / same_k of `a` from its
+// members' shapes.  Host side.
+inline void finish_group(GemmArgs& a)
+{
+    int g = 0, kmax = 0, same = 1;
+    for (int i = 0; i < a.nmem; ++i) {
+        a.mem[i].g0 = g;
+        g += a.mem[i].n_out / 128;
+        if (a.mem[i].k_in > kmax) kmax = a.mem[i].k_in;
+        if (a.mem[i].k_in != a.mem[0].k_in) same = 0;
+    }
+    a.n_out = 128 * g;
+    a.k_max = kmax;
+    a.same_k = same;
+}
+
 #ifdef __CUDACC__
-// The sibling holding group output block g, and g's block index inside it.
-// Unrolled over the fixed-size table (no dynamically indexed parameters).
-struct SibView {
+// The member holding a group output block or work unit, with the block's
+// index inside it.  Selected by unrolled compares over the fixed-size table
+// (no dynamically indexed kernel parameters).
+struct MemView {
+    const uint16_t* x;
+    const uint16_t* su;
     const uint32_t* packed;
     const uint16_t* scale;
     const uint16_t* sv;
     void* y;
-    int n_out;
-    int gl;
+    int k_in, n_out;
+    int g0;
+    long long u0;
+    long long xt0;
+    int gl;                   // block index inside the member (member_of_block)
 };
-__device__ __forceinline__ SibView sibling_of(const GemmArgs& a, int g)
+__device__ __forceinline__ MemView view_of(const Member& t)
 {
-    SibView v{a.sib[0].packed, a.sib[0].scale, a.sib[0].sv, a.sib[0].y, a.sib[0].n_out, g};
+    return MemView{t.x, t.su, t.packed, t.scale, t.sv, t.y, t.k_in, t.n_out, t.g0, t.u0, t.xt0, 0};
+}
+__device__ __forceinline__ MemView member_of_block(const GemmArgs& a, int g)
+{
+    MemView v = view_of(a.mem[0]);
 #pragma unroll
-    for (int t = 1; t < kMaxSiblings; ++t) {
-        if (t < a.nsib && g >= a.sib[t].g0) {
-            v = SibView{a.sib[t].packed, a.sib[t].scale, a.sib[t].sv, a.sib[t].y, a.sib[t].n_out, g - a.sib[t].g0};
-        }
-    }
+    for (int t = 1; t < kMaxMembers; ++t)
+        if (t < a.nmem && g >= a.mem[t].g0) v = view_of(a.mem[t]);
+    v.gl = g - v.g0;
+    return v;
+}
+__device__ __forceinline__ MemView member_of_unit(const GemmArgs& a, long long u)
+{
+    MemView v = view_of(a.mem[0]);
+#pragma unroll
+    for (int t = 1; t < kMaxMembers; ++t)
+        if (t < a.nmem && u >= a.mem[t].u0) v = view_of(a.mem[t]);
     return v;
 }
 #endif
@@ -80,8 +122,10 @@ cudaError_t once_per_device(std::atomic<int> (&done)[kMaxDevices], F&& setup)
     return e;
 }
 
-// Single-row product on CUDA cores (gemv_m1.cu).
+// Single-row product on CUDA cores (gemv_m1.cu).  The workspace of a group
+// depends on its total width and its total work (tile rows).
 size_t m1_workspace_bytes(int k_in, int n_out, int bits);
+size_t m1_group_workspace_bytes(const GemmArgs& a);
 cudaError_t launch_gemv_m1(const GemmArgs& a, cudaStream_t stream);
 
 // Tensor-core path (2..32 rows): CTA count (planned), workspace size,
@@ -89,6 +133,7 @@ cudaError_t launch_gemv_m1(const GemmArgs& a, cudaStream_t stream);
 // kernel, launched as clusters of the CTAs that share an output block).
 int tc_ctas(int m, int k_in, int n_out, int bits);
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits);
+size_t tc_group_workspace_bytes(const GemmArgs& a);
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream);
 
 // Many-row path (gemm_large.cu): decode once into the tensor-core operand

@@ -409,21 +409,22 @@ cudaError_t launch_decode_image(const uint32_t* packed, int k_in, int n_out, uin
 
 cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
 {
-    const Sibling& sb = a.sib[0];
+    const Member& sb = a.mem[0];                 // one product per call
+    const int k_in = sb.k_in;
     const int nb = large_tile_rows(a.m, a.n_out);
     const int m_pad = (a.m + nb - 1) / nb * nb;
     uint8_t* image = a.ws + kWsHeader;
-    uint8_t* xt = image + (size_t)a.k_in * a.n_out * 2;
+    uint8_t* xt = image + (size_t)k_in * a.n_out * 2;
 
     cudaError_t e = cudaErrorInvalidValue;
     switch (a.bits) {
-        case 2: e = launch_decode_image<2>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
-        case 3: e = launch_decode_image<3>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
-        case 4: e = launch_decode_image<4>(sb.packed, a.k_in, a.n_out, image, stream, a.pdl); break;
+        case 2: e = launch_decode_image<2>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
+        case 3: e = launch_decode_image<3>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
+        case 4: e = launch_decode_image<4>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
     }
     if (e != cudaSuccess) return e;
     {
-        const long long items = (long long)m_pad * ((a.k_in / 128 + 3) / 4);
+        const long long items = (long long)m_pad * ((k_in / 128 + 3) / 4);
         cudaLaunchConfig_t cfg = {};
         cudaLaunchAttribute attr[1];
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -433,8 +434,8 @@ cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
         cfg.stream = stream;
         cfg.attrs = attr;
         cfg.numAttrs = a.pdl ? 1 : 0;
-        e = cudaLaunchKernelEx(&cfg, xt_tiled_prepass_kernel, reinterpret_cast<const __half*>(a.x),
-                               reinterpret_cast<const __half*>(a.su), a.m, m_pad, a.k_in, nb, xt);
+        e = cudaLaunchKernelEx(&cfg, xt_tiled_prepass_kernel, reinterpret_cast<const __half*>(sb.x),
+                               reinterpret_cast<const __half*>(sb.su), a.m, m_pad, k_in, nb, xt);
         if (e != cudaSuccess) return e;
     }
     LgParams prm;
@@ -446,12 +447,12 @@ cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
     prm.status = reinterpret_cast<uint32_t*>(a.ws);
     prm.y_fp32 = a.y_fp32;
     prm.m = a.m;
-    prm.k_in = a.k_in;
+    prm.k_in = k_in;
     prm.n_out = a.n_out;
     prm.J = m_pad / nb;
     {
         // L2 working set of a wave of tiles in each order (bytes): keep the smaller
-        const double image = 2.0 * a.k_in * a.n_out, xtb = 2.0 * m_pad * a.k_in;
+        const double image = 2.0 * k_in * a.n_out, xtb = 2.0 * m_pad * k_in;
         const double wave = 148.0;                 // about one tile per SM in flight
         const double G = a.n_out / 128, J = prm.J;
         const double g_fast = image + xtb * (wave / G < J ? wave / G : J) / J;

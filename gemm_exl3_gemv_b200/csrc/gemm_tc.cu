@@ -104,10 +104,9 @@ struct TcParams {
     float* part;            // stream-K partial sums, [slot][NT][128]
     uint32_t* counters;     // stream-K arrival counters, per output block
     uint32_t* status;       // workspace status word
-    int C;                  // 128-row input blocks (units per output block)
     int S;                  // cluster size (CTAs per output block), 0: stream-K
     int P;                  // stream-K CTAs
-    long long U;            // units = G * C
+    long long U;            // units: sum over members of blocks x 128-row input blocks
     uint32_t two16;         // 2^16, passed at run time (keeps a multiply on the FMA pipe)
 };
 
@@ -184,7 +183,7 @@ __device__ __forceinline__ void reduce_segments(const float* part, int g, int p_
 // channels 4*lane .. +3) times scale, output rotation, signs, store.
 __device__ __forceinline__ void finish_row_regs(const GemmArgs& a, int g, int mm, const float (&z)[4], int lane)
 {
-    const SibView sib = sibling_of(a, g);                 // the matrix holding block g
+    const MemView sib = member_of_block(a, g);            // the matrix holding block g
     const int n0 = 128 * sib.gl + 4 * lane;
     const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
     const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
@@ -233,14 +232,17 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
 
     const GemmArgs& a = prm.a;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int S = prm.S, C = prm.C;
+    const int S = prm.S;
     const int p = blockIdx.x;
-    // this CTA's units [b0, b1) in block-major order
+    // this CTA's units [b0, b1) in the group's block-major order
     long long b0, b1;
     if (S > 0) {
         const int gc = p / S, rc = p % S;
-        b0 = (long long)gc * C + (long long)rc * C / S;
-        b1 = (long long)gc * C + (long long)(rc + 1) * C / S;
+        const MemView cm = member_of_block(a, gc);
+        const int C = cm.k_in / 128;
+        const long long ublk = cm.u0 + (long long)cm.gl * C;
+        b0 = ublk + (long long)rc * C / S;
+        b1 = ublk + (long long)(rc + 1) * C / S;
     } else {
         b0 = (long long)p * prm.U / prm.P;
         b1 = (long long)(p + 1) * prm.U / prm.P;
@@ -276,13 +278,13 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         const long long allowed = inject ? (long long)inject - 1 : (b1 - b0);
         if (lane == 0) {
             int kk = 0;
-            int c = (int)(b0 % C);
             for (long long u = b0; u < b1 && kk < allowed; ++u, ++kk) {
                 const int s = kk & (kBStages - 1);
                 if (kk >= kBStages && !wait_or_abort(&bempty[s], (uint32_t)(kk / kBStages - 1) & 1u, abort_flag)) break;
+                const MemView um = member_of_unit(a, u);
+                const int c = (int)((u - um.u0) % (um.k_in / 128));
                 mbar_arrive_expect_tx(&bfull[s], L::BUNIT);
-                bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
-                if (++c == C) c = 0;
+                bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + um.xt0 + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
             }
             // every issued copy lands before the CTA can exit (a no-op wait in
             // a normal run: the decoders have consumed them)
@@ -314,14 +316,17 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         int kk = 0;                                              // CTA unit counter (stages, parities)
         int seg = 0;
         for (long long u0 = b0; u0 < b1; ++seg) {
-            const int g = (int)(u0 / C);
-            const int c0 = (int)(u0 - (long long)g * C);
-            const long long u1 = ((long long)(g + 1) * C < b1) ? (long long)(g + 1) * C : b1;
+            const MemView sib = member_of_unit(a, u0);                 // the matrix holding unit u0
+            const int C = sib.k_in / 128;                              // units per block of this matrix
+            const int gl = (int)((u0 - sib.u0) / C);
+            const int g = sib.g0 + gl;                                 // group block index
+            const long long ublk = sib.u0 + (long long)gl * C;         // the block's first unit
+            const int c0 = (int)(u0 - ublk);
+            const long long u1 = (ublk + C < b1) ? ublk + C : b1;
             const int nseg = (int)(u1 - u0);
-            const SibView sib = sibling_of(a, g);                      // the matrix holding block g
             const int tiles_n = sib.n_out / 16;
             const uint32_t* src =
-                sib.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)sib.gl) * TW + (size_t)lane * QW;
+                sib.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
             const size_t unit_step = (size_t)8 * tiles_n * TW;    // words between consecutive units
             bool ok = true;                                      // warp-uniform
             // decode the segment's unit k (the CTA's kk-th) from `wds` into A
@@ -408,8 +413,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             named_bar(1, 32 * kDec);
             bool finish = true;
             if (nseg < C) {
-                const int p_first = cta_of_unit((long long)g * C, prm.P, prm.U);
-                const int p_last = cta_of_unit((long long)(g + 1) * C - 1, prm.P, prm.U);
+                const int p_first = cta_of_unit(ublk, prm.P, prm.U);
+                const int p_last = cta_of_unit(ublk + C - 1, prm.P, prm.U);
                 float4* myslot = reinterpret_cast<float4*>(prm.part + (size_t)(p + g) * NT * 128);
                 const float4* z4s = reinterpret_cast<const float4*>(zsm);
                 for (int f = threadIdx.x; f < a.m * 32; f += 32 * kDec) __stcg(myslot + f, z4s[f]);
@@ -486,24 +491,47 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
 // xt = H(su .* x) / sqrt(128) for rows 0..NT-1 (zero rows past m), written in
 // the B-operand layout: 64-row chunks of NT x 128 bytes, rows of 8 x 16-byte
 // pieces swizzled by (row & 7), and inside each 16-row group k = 4q + r
-// placed at position 8(r >> 1) + 4(r & 1) + q.
+// placed at position 8(r >> 1) + 4(r & 1) + q.  One warp item = (member,
+// row, 128-block); a sibling group (shared x) rotates member 0's x only.
 template <int NT>
-__global__ void __launch_bounds__(256) xt_prepass_kernel(const __half* __restrict__ x, const __half* __restrict__ su,
-                                                         int m_rows, int k_in, uint8_t* __restrict__ xt)
+__global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8_t* __restrict__ xt_base)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dep_launch();                 // the product kernel may start its prologue
     grid_dep_wait();                   // x and the workspace only after the previous kernel
+    long long item = (long long)blockIdx.x * 8 + warp;
+    // the member of this item: members in order, NT * (k_in / 128) items each
+    const __half* x = reinterpret_cast<const __half*>(a.mem[0].x);
+    const __half* su = reinterpret_cast<const __half*>(a.mem[0].su);
+    int k_in = a.mem[0].k_in;
+    long long xt0 = a.mem[0].xt0;
+    bool found = false;
+    const int nm = a.shared_x ? 1 : a.nmem;
+#pragma unroll
+    for (int t = 0; t < kMaxMembers; ++t) {
+        if (t < nm && !found) {
+            const long long cnt = (long long)NT * (a.mem[t].k_in / 128);
+            if (item < cnt) {
+                found = true;
+                x = reinterpret_cast<const __half*>(a.mem[t].x);
+                su = reinterpret_cast<const __half*>(a.mem[t].su);
+                k_in = a.mem[t].k_in;
+                xt0 = a.mem[t].xt0;
+            } else {
+                item -= cnt;
+            }
+        }
+    }
+    if (!found) return;
     const int nblk = k_in / 128;
-    const long long item = (long long)blockIdx.x * 8 + warp;
-    if (item >= (long long)NT * nblk) return;
     const int m = (int)(item / nblk), b = (int)(item % nblk);
+    uint8_t* xt = const_cast<uint8_t*>(xt_base) + xt0;
     // lane holds elements i = (lane & 3) | (e << 2) | ((lane >> 2) << 4)
     float v[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
         const int k = 128 * b + ((lane & 3) | (e << 2) | ((lane >> 2) << 4));
-        v[e] = (m < m_rows) ? __half2float(x[(size_t)m * k_in + k]) * __half2float(su[k]) : 0.f;
+        v[e] = (m < a.m) ? __half2float(x[(size_t)m * k_in + k]) * __half2float(su[k]) : 0.f;
     }
     fwht128_warp(v);   // the transform factors over index bits: any bit-to-(lane, e) map works
     const int tr = 8 * b + (lane >> 2);
@@ -519,20 +547,43 @@ int nt_for(int m) { return m <= 16 ? 16 : 32; }
 
 size_t xt_offset(int G) { return align_up(ws_counter_off() + 4 * (size_t)G, 1024); }
 
+// Units of the group (sum over members of blocks x 128-row input blocks).
+long long group_units(const GemmArgs& a)
+{
+    long long U = 0;
+    for (int i = 0; i < a.nmem; ++i) U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / 128);
+    return U;
+}
+
+// Bytes of rotated input: one k_in x NT fp16 operand per distinct input.
+size_t xt_bytes(const GemmArgs& a, int NT)
+{
+    if (a.shared_x) return (size_t)a.mem[0].k_in * NT * 2;
+    size_t b = 0;
+    for (int i = 0; i < a.nmem; ++i) b += (size_t)a.mem[i].k_in * NT * 2;
+    return b;
+}
+
 // stream-K CTA count: one wave (two CTAs per SM), at most 8 CTAs per output
 // block on average (the last CTA of a block reads every partial of it), at
 // most one CTA per unit
-int sk_ctas(int k_in, int n_out)
+int sk_ctas(int G, long long U)
 {
-    const long long G = n_out / 128, U = G * (k_in / 128);
     long long p = (long long)kSms * kCtasPerSm;
-    if (p > 8 * G) p = 8 * G;
+    if (p > 8LL * G) p = 8LL * G;
     if (p > U) p = U;
     if (p < 1) p = 1;
     return (int)p;
 }
 
-size_t part_offset(int k_in, int n_out, int NT) { return align_up(xt_offset(n_out / 128) + (size_t)k_in * NT * 2, 256); }
+size_t part_offset(const GemmArgs& a, int NT) { return align_up(xt_offset(a.n_out / 128) + xt_bytes(a, NT), 256); }
+
+size_t group_ws_bytes(const GemmArgs& a, int NT)
+{
+    // the stream-K partial slots are always reserved (either cut may be chosen)
+    const int G = a.n_out / 128;
+    return part_offset(a, NT) + (size_t)(sk_ctas(G, group_units(a)) + G) * NT * 128 * sizeof(float);
+}
 
 // Stand-in with the product kernel's block size and shared memory but
 // nothing else, for the cluster-occupancy query: for the product kernel
@@ -577,7 +628,7 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
         const double segs = (P % G == 0) ? 1.0 : (double)((per - 1) / C + 2);
         return (double)per + 0.3 * (double)P / G + kSegCost * segs + kGlobalRed;
     };
-    TcPlan best{0, sk_ctas(k_in, n_out)};
+    TcPlan best{0, sk_ctas(G, U)};
     double best_cost = cost_sk(best.P);
     // aligned stream-K: S' CTAs per block (S' <= 8 keeps P within the workspace's partial slots)
     for (int s2 = 2; s2 <= 8 && (long long)s2 * G <= (long long)kSms * kCtasPerSm && s2 <= C; ++s2) {
@@ -617,23 +668,33 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
 }
 
 template <int BITS, int NT>
-cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
+cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
 {
     using L = TcLayout<NT>;
+    // member units and rotated-input offsets of the group
+    {
+        long long U = 0, xo = 0;
+        for (int i = 0; i < a.nmem; ++i) {
+            a.mem[i].u0 = U;
+            U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / 128);
+            a.mem[i].xt0 = a.shared_x ? 0 : xo;
+            xo += (long long)a.mem[i].k_in * NT * 2;
+        }
+    }
     TcParams prm;
     prm.a = a;
     const int G = a.n_out / 128;
-    prm.C = a.k_in / 128;
-    prm.U = (long long)G * prm.C;
+    prm.U = group_units(a);
     prm.two16 = 0x10000u;
     uint8_t* ws = a.ws;
     prm.status = reinterpret_cast<uint32_t*>(ws);
     prm.counters = reinterpret_cast<uint32_t*>(ws + ws_counter_off());
     const size_t xt_off = xt_offset(G);
     prm.xt = ws + xt_off;
-    prm.part = reinterpret_cast<float*>(ws + part_offset(a.k_in, a.n_out, NT));
+    prm.part = reinterpret_cast<float*>(ws + part_offset(a, NT));
 
-    const long long items = (long long)NT * (a.k_in / 128);
+    long long items = 0;
+    for (int i = 0; i < (a.shared_x ? 1 : a.nmem); ++i) items += (long long)NT * (a.mem[i].k_in / 128);
     cudaLaunchAttribute pdl_attr;
     pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr.val.programmaticStreamSerializationAllowed = 1;
@@ -644,8 +705,7 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
         pcfg.stream = stream;
         pcfg.attrs = &pdl_attr;
         pcfg.numAttrs = a.pdl ? 1 : 0;
-        cudaError_t e = cudaLaunchKernelEx(&pcfg, xt_prepass_kernel<NT>, reinterpret_cast<const __half*>(a.x),
-                                           reinterpret_cast<const __half*>(a.su), a.m, a.k_in, ws + xt_off);
+        cudaError_t e = cudaLaunchKernelEx(&pcfg, xt_prepass_kernel<NT>, a, (const uint8_t*)(ws + xt_off));
         if (e != cudaSuccess) return e;
     }
     cudaError_t e = cudaGetLastError();
@@ -665,24 +725,32 @@ cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
     });
     if (e != cudaSuccess) return e;
 
-    // plan decided once per shape (host-side occupancy queries), then cached
-    static std::mutex mu;
-    static long long cache_key[32] = {};
-    static TcPlan cache_val[32];
-    static int cache_next = 0;
-    const long long key = (long long)a.k_in * 1000003LL + a.n_out;
-    TcPlan pl{-1, 0};
-    {
-        std::lock_guard<std::mutex> lock(mu);
-        for (int i = 0; i < 32; ++i)
-            if (cache_key[i] == key) pl = cache_val[i];
-    }
-    if (pl.S < 0) {
-        pl = choose_plan(a.k_in, a.n_out, L::total);
-        std::lock_guard<std::mutex> lock(mu);
-        cache_key[cache_next] = key;
-        cache_val[cache_next] = pl;
-        cache_next = (cache_next + 1) % 32;
+    TcPlan pl{0, sk_ctas(G, prm.U)};
+    if (a.same_k) {
+        // one block length: plan decided once per shape (host-side occupancy
+        // queries), then cached.  Groups of several lengths take stream-K.
+        static std::mutex mu;
+        static long long cache_key[32] = {};
+        static TcPlan cache_val[32];
+        static int cache_next = 0;
+        const int k_in = a.mem[0].k_in;
+        const long long key = (long long)k_in * 1000003LL + a.n_out;
+        bool hit = false;
+        {
+            std::lock_guard<std::mutex> lock(mu);
+            for (int i = 0; i < 32; ++i)
+                if (cache_key[i] == key) {
+                    pl = cache_val[i];
+                    hit = true;
+                }
+        }
+        if (!hit) {
+            pl = choose_plan(k_in, a.n_out, L::total);
+            std::lock_guard<std::mutex> lock(mu);
+            cache_key[cache_next] = key;
+            cache_val[cache_next] = pl;
+            cache_next = (cache_next + 1) % 32;
+        }
     }
     prm.S = pl.S;
     prm.P = pl.S > 0 ? 0 : pl.P;
@@ -711,15 +779,22 @@ int tc_ctas(int m, int k_in, int n_out, int bits)
 {
     (void)m;
     (void)bits;
-    return sk_ctas(k_in, n_out);
+    return sk_ctas(n_out / 128, (long long)(n_out / 128) * (k_in / 128));
 }
+
+size_t tc_group_workspace_bytes(const GemmArgs& a) { return group_ws_bytes(a, nt_for(a.m)); }
 
 size_t tc_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
-    (void)bits;
-    const int NT = nt_for(m);
-    // the stream-K partial slots are always reserved (either cut may be chosen)
-    return part_offset(k_in, n_out, NT) + (size_t)(sk_ctas(k_in, n_out) + n_out / 128) * NT * 128 * sizeof(float);
+    GemmArgs a = {};
+    a.m = m;
+    a.bits = bits;
+    a.nmem = 1;
+    a.shared_x = 1;
+    a.mem[0].k_in = k_in;
+    a.mem[0].n_out = n_out;
+    finish_group(a);
+    return group_ws_bytes(a, nt_for(m));
 }
 
 cudaError_t launch_gemm_tc(const GemmArgs& a, cudaStream_t stream)

@@ -116,8 +116,7 @@ __device__ __forceinline__ void tile_row(const uint32_t (&w)[2 * BITS], const ui
 // p + g (unique: ranges are monotone).
 struct M1Plan {
     int P;            // CTAs
-    int T;            // tile rows per channel block (k_in / 16)
-    long long U;      // units G * T
+    long long U;      // units: sum over the group's members of blocks x tile rows
     int kb_max;       // 128-row input blocks one segment can touch
 };
 
@@ -139,7 +138,6 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int p = blockIdx.x;
-    const int T = pl.T;
     const long long b0 = (long long)p * pl.U / pl.P, b1 = (long long)(p + 1) * pl.U / pl.P;
     const int q = lane & 3;
     const int src_prev = (lane & ~3) | ((q + 3) & 3);
@@ -149,10 +147,14 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     bool first_seg = true;
 
     for (long long u = b0; u < b1;) {
-        // ---- segment: block g, tile rows [r0, r1) ----
-        const int g = (int)(u / T);
-        const int r0 = (int)(u - (long long)g * T);
-        const int r1 = (int)(((long long)(g + 1) * T < b1 ? (long long)(g + 1) * T : b1) - (long long)g * T);
+        // ---- segment: block g (group numbering) = block gl of member mv, tile rows [r0, r1) ----
+        const MemView mv = member_of_unit(a, u);
+        const int T = mv.k_in / 16;                                    // tile rows per block of this member
+        const int gl = (int)((u - mv.u0) / T);
+        const int g = mv.g0 + gl;
+        const long long ublk = mv.u0 + (long long)gl * T;              // the block's first unit
+        const int r0 = (int)(u - ublk);
+        const int r1 = (int)((ublk + T < b1 ? ublk + T : b1) - ublk);
         u += r1 - r0;
         const int kb_lo = r0 >> 3, kb_hi = (r1 + 7) >> 3;             // 128-row input blocks touched
         const int nrow = r1 - r0;
@@ -160,10 +162,9 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         size_t row_step;                                               // words between a warp's rows
         const uint32_t* src;
         {
-            const SibView sw = sibling_of(a, g);                       // the matrix holding block g
-            const int tiles_n = sw.n_out / 16;
+            const int tiles_n = mv.n_out / 16;
             row_step = (size_t)kM1Warps * tiles_n * TW;
-            src = sw.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)sw.gl) * TW + (size_t)lane * QW;
+            src = mv.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
         }
         uint32_t wa[QW], wb[QW];
         if (nw > 0) load_lane_words<BITS>(wa, src);                       // in flight during the rotation
@@ -174,8 +175,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         // input rotation of the touched blocks: xxs[k - 128 kb_lo] = (xt, xt)
         for (int kb = kb_lo + warp; kb < kb_hi; kb += kM1Warps) {
             const int col = kb * 128 + 4 * lane;
-            const uint2 raw = *reinterpret_cast<const uint2*>(a.x + col);
-            const uint2 sraw = *reinterpret_cast<const uint2*>(a.su + col);
+            const uint2 raw = *reinterpret_cast<const uint2*>(mv.x + col);
+            const uint2 sraw = *reinterpret_cast<const uint2*>(mv.su + col);
             const float2 x0 = __half22float2(as_h2(raw.x)), x1 = __half22float2(as_h2(raw.y));
             const float2 s0 = __half22float2(as_h2(sraw.x)), s1 = __half22float2(as_h2(sraw.y));
             float v[4] = {x0.x * s0.x, x0.y * s0.y, x1.x * s1.x, x1.y * s1.y};
@@ -236,8 +237,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
 
         // ---- a block split over several CTAs: the last to arrive finishes it ----
         if (nrow < T) {
-            const int p_first = m1_cta_of_unit((long long)g * T, pl.P, pl.U);
-            const int p_last = m1_cta_of_unit((long long)(g + 1) * T - 1, pl.P, pl.U);
+            const int p_first = m1_cta_of_unit(ublk, pl.P, pl.U);
+            const int p_last = m1_cta_of_unit(ublk + T - 1, pl.P, pl.U);
             if (threadIdx.x < 128) __stcg(part + (size_t)(p + g) * 128 + threadIdx.x, z);
             __threadfence();
             __syncthreads();
@@ -276,8 +277,8 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
 
         // ---- epilogue (warp 0): scale, output rotation, signs, store ----
         if (warp == 0) {
-            const SibView sib = sibling_of(a, g);
-            const int n0 = 128 * sib.gl + 4 * lane;
+            const MemView sib = mv;
+            const int n0 = 128 * gl + 4 * lane;
             const float4 z4 = *reinterpret_cast<const float4*>(red + 4 * lane);
             const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
             const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
@@ -299,20 +300,27 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     }
 }
 
-M1Plan m1_plan(int k_in, int n_out, int bits)
+// Units of member i start at u0 = the tile rows of the members before it.
+// Sets a.mem[i].u0 (host side) and returns the plan.
+M1Plan m1_plan(GemmArgs& a)
 {
-    const int G = n_out / 128;
-    const int per_sm = bits == 2 ? kM1MinBlocks<2> : bits == 3 ? kM1MinBlocks<3> : kM1MinBlocks<4>;
+    const int per_sm = kM1MinBlocks<3>;
+    long long U = 0;
+    for (int i = 0; i < a.nmem; ++i) {
+        a.mem[i].u0 = U;
+        U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / 16);
+    }
+    const int G = a.n_out / 128;
     M1Plan pl;
-    pl.T = k_in / 16;
-    pl.U = (long long)G * pl.T;
+    pl.U = U;
     const long long slots = (long long)kSms * per_sm;   // one wave of resident CTAs
-    // Give every block the same whole number of CTAs, so that no range
-    // straddles two blocks (one segment per CTA: the per-segment costs --
-    // input rotation, reduction, arrival -- are paid once), unless that
-    // leaves more than 15 % of the slots idle; then cut evenly across blocks
-    // (stream-K).
-    long long P = G <= slots ? (long long)G * (slots / G) : slots;
+    // When every block has the same length (one k_in), give every block the
+    // same whole number of CTAs, so that no range straddles two blocks (one
+    // segment per CTA: the per-segment costs -- input rotation, reduction,
+    // arrival -- are paid once), unless that leaves more than 15 % of the
+    // slots idle; then, and for groups of several lengths, cut evenly across
+    // blocks (stream-K).
+    long long P = (a.same_k && G <= slots) ? (long long)G * (slots / G) : slots;
     if (20 * P < 17 * slots) P = slots;                 // whole-block split would idle >15 % of the slots
     if (P > pl.U / kM1Warps) P = pl.U / kM1Warps;       // at least one tile row per warp
     const long long rows_cap = 1024;                    // bounds the rotated input kept in shared memory
@@ -342,9 +350,9 @@ template <int BITS>
 constexpr int kAltEvery = BITS == 3 ? EXL3_M1_ALT3 : EXL3_M1_ALT24;
 
 template <int BITS>
-cudaError_t launch_m1_t(const GemmArgs& a, cudaStream_t stream)
+cudaError_t launch_m1_t(GemmArgs a, cudaStream_t stream)
 {
-    const M1Plan pl = m1_plan(a.k_in, a.n_out, a.bits);
+    const M1Plan pl = m1_plan(a);
     const size_t smem = m1_smem_bytes(pl);
     auto kern = gemv_m1_kernel<BITS, kAltEvery<BITS>>;
     static std::atomic<int> configured[kMaxDevices];
@@ -370,10 +378,23 @@ cudaError_t launch_m1_t(const GemmArgs& a, cudaStream_t stream)
 
 }  // namespace
 
+size_t m1_group_workspace_bytes(const GemmArgs& a0)
+{
+    GemmArgs a = a0;
+    const M1Plan pl = m1_plan(a);
+    return ws_part_off(a.n_out) + (size_t)(pl.P + a.n_out / 128) * 128 * sizeof(float);
+}
+
 size_t m1_workspace_bytes(int k_in, int n_out, int bits)
 {
-    const M1Plan pl = m1_plan(k_in, n_out, bits);
-    return ws_part_off(n_out) + (size_t)(pl.P + n_out / 128) * 128 * sizeof(float);
+    GemmArgs a = {};
+    a.m = 1;
+    a.bits = bits;
+    a.nmem = 1;
+    a.mem[0].k_in = k_in;
+    a.mem[0].n_out = n_out;
+    finish_group(a);
+    return m1_group_workspace_bytes(a);
 }
 
 cudaError_t launch_gemv_m1(const GemmArgs& a, cudaStream_t stream)

@@ -29,7 +29,7 @@ EXL3_ERR_TIMEOUT = 7
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",
            "exl3_workspace_status", "exl3_kernel_launches", "exl3_decode_tiles", "exl3_hadamard128", "exl3_gemv",
            "exl3_gemm_small_m", "exl3_gemm_siblings", "exl3_large_m_workspace_bytes", "exl3_gemm_large_m",
-           "exl3_gemv_noalloc")
+           "exl3_gemv_noalloc", "exl3_grouped_workspace_bytes", "exl3_gemm_grouped")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"libexl3.so not built ({LIB_PATH}); run `python -m gemm_exl3_gemv_b200.build`")
@@ -71,6 +71,18 @@ lib.exl3_large_m_workspace_bytes.restype = _Z
 lib.exl3_gemm_large_m.argtypes = [_I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]
 lib.exl3_gemm_large_m.restype = _I
 lib.exl3_gemv_noalloc.restype = _I
+
+
+class Problem(ctypes.Structure):
+    """exl3_problem_t: one member of a grouped call (device pointers)."""
+    _fields_ = [("x", _P), ("su", _P), ("packed", _P), ("scale", _P), ("sv", _P), ("y", _P),
+                ("k_in", _I), ("n_out", _I)]
+
+
+lib.exl3_grouped_workspace_bytes.argtypes = [_I, ctypes.POINTER(Problem), _I, _I]
+lib.exl3_grouped_workspace_bytes.restype = _Z
+lib.exl3_gemm_grouped.argtypes = [_I, ctypes.POINTER(Problem), _I, _I, _I, _P, _Z, _P]
+lib.exl3_gemm_grouped.restype = _I
 
 
 class Exl3Error(RuntimeError):
@@ -203,3 +215,44 @@ def gemm_large(x: torch.Tensor, packed: torch.Tensor, scale: torch.Tensor, su: t
     _check(st, "exl3_gemm_large_m")
     return out
 
+
+
+def grouped_workspace_bytes(m: int, shapes, bits: int) -> int:
+    """Workspace of a grouped call for members of shapes [(k_in, n_out), ...]."""
+    arr = (Problem * len(shapes))()
+    for i, (k, n) in enumerate(shapes):
+        arr[i] = Problem(None, None, None, None, None, None, int(k), int(n))
+    return int(lib.exl3_grouped_workspace_bytes(m, arr, len(shapes), bits))
+
+
+def grouped_kernel_launches(m: int) -> int:
+    """Kernel launches of one grouped call: the product (m = 1), or the
+    rotation pre-pass and the product (m >= 2)."""
+    return 1 if m == 1 else 2
+
+
+def gemm_grouped(problems, bits: int, fp32: bool = False, workspace: Optional[torch.Tensor] = None,
+                 stream=None):
+    """Products of independent problems in one pass.  `problems` is a list of
+    (x, packed, scale, su, sv, y) device tensors, x of shape (m, k_in) (or
+    (k_in,) for m = 1) and y of shape (m, n_out); returns the list of y."""
+    arr = (Problem * len(problems))()
+    m = None
+    shapes = []
+    for i, (x, packed, scale, su, sv, y) in enumerate(problems):
+        x2 = x.reshape(1, -1) if x.dim() == 1 else x
+        if m is None:
+            m = x2.shape[0]
+        k_in, n_out = x2.shape[1], scale.shape[0]
+        shapes.append((k_in, n_out))
+        arr[i] = Problem(x2.data_ptr(), su.data_ptr(), packed.data_ptr(), scale.data_ptr(), sv.data_ptr(),
+                         y.data_ptr(), int(k_in), int(n_out))
+    if workspace is None:
+        n = grouped_workspace_bytes(m, shapes, bits)
+        if n == 0:
+            raise Exl3Error(EXL3_ERR_UNSUPPORTED, "exl3_grouped_workspace_bytes")
+        workspace = torch.zeros(n, dtype=torch.uint8, device=problems[0][0].device)
+    st = lib.exl3_gemm_grouped(m, arr, len(problems), int(fp32), bits, _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "exl3_gemm_grouped")
+    return [p[5] for p in problems]

@@ -125,18 +125,27 @@ class MatrixInputs:
     sv: np.ndarray                 # fp16 +-1, N_out
 
 
-def small_inputs(spec: MatrixSpec):
-    """scale, x, su, sv for a matrix (numpy PCG64 seeded by [seed, layer, index])."""
+# Chained runs (a layer's output is the next layer's input) divide the scales
+# by this factor, so that activations stay near unit size along a deep chain
+# instead of growing by about that factor per product.
+CHAIN_SCALE_DIV = 1.3
+
+
+def small_inputs(spec: MatrixSpec, chain: bool = False):
+    """scale, x, su, sv for a matrix (numpy PCG64 seeded by [seed, layer, index]).
+    chain=True: the scales of a chained run (same draw, divided by
+    CHAIN_SCALE_DIV before the fp16 rounding)."""
     rng = np.random.default_rng([spec.seed, spec.layer, spec.index])
-    scale = (rng.uniform(0.5, 1.5, spec.n_out) / np.sqrt(spec.k_in)).astype(np.float16)
+    div = np.sqrt(spec.k_in) * (CHAIN_SCALE_DIV if chain else 1.0)
+    scale = (rng.uniform(0.5, 1.5, spec.n_out) / div).astype(np.float16)
     x = rng.standard_normal((spec.m, spec.k_in)).astype(np.float16)
     su = np.where(rng.integers(0, 2, spec.k_in) == 0, 1.0, -1.0).astype(np.float16)
     sv = np.where(rng.integers(0, 2, spec.n_out) == 0, 1.0, -1.0).astype(np.float16)
     return scale, x, su, sv
 
 
-def make_inputs(spec: MatrixSpec, with_packed: bool = True) -> MatrixInputs:
-    scale, x, su, sv = small_inputs(spec)
+def make_inputs(spec: MatrixSpec, with_packed: bool = True, chain: bool = False) -> MatrixInputs:
+    scale, x, su, sv = small_inputs(spec, chain)
     packed = splitmix64_words_np(spec.stream_id, 0, spec.n_words) if with_packed else None
     return MatrixInputs(spec, packed, scale, x, su, sv)
 

@@ -158,6 +158,12 @@ EXL3_API int exl3_gemv(const uint16_t *x, const uint32_t *packed, const uint16_t
  *   exl3_workspace_bytes(m, k_in, n_out, bits).
  * Deterministic as exl3_gemv.  Different m may use different kernels, which
  * agree within rounding, not bitwise.
+ * Timeouts (m >= 2): every wait inside the kernel is bounded (2 s).  If one
+ * runs out the call has ALREADY returned EXL3_OK and y is not valid; nothing
+ * reports it until exl3_workspace_status(workspace, stream), which
+ * synchronises.  Callers that cannot rule out a stalled GPU poll it.  The
+ * same holds for exl3_gemm_siblings and exl3_gemm_grouped at m >= 2 and for
+ * exl3_gemm_large_m.  The single-row kernel (m = 1) never waits on anything.
  */
 EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
                       const uint16_t *scale, const uint16_t *su, const uint16_t *sv,
@@ -178,7 +184,8 @@ EXL3_API int exl3_gemm_small_m(int m, const uint16_t *x, const uint32_t *packed,
  *     element, rounded up to the row tile), 256-byte aligned; its first word
  *     is the status word exl3_workspace_status reads.  No zero-fill needed.
  * Each output is one accumulator's fixed-order sum: repeated calls are
- * bitwise identical.
+ * bitwise identical.  A bounded wait that runs out is reported only by
+ * exl3_workspace_status (the call itself has returned EXL3_OK).
  */
 EXL3_API size_t exl3_large_m_workspace_bytes(int m, int k_in, int n_out, int bits);
 EXL3_API int exl3_gemm_large_m(int m, const uint16_t *x, const uint32_t *packed, const uint16_t *scale,
@@ -215,6 +222,46 @@ typedef struct exl3_matrix {
 EXL3_API int exl3_gemm_siblings(int m, const uint16_t *x, const uint16_t *su, const exl3_matrix_t *mats,
                                 int n_mats, int y_fp32, int k_in, int bits, void *workspace, size_t ws_bytes,
                                 void *stream);
+
+/*
+ * exl3_gemm_grouped -- the products of up to 8 INDEPENDENT problems in one
+ * pass: y_i = sv_i .* H(scale_i .* (H(su_i .* x_i) W_i)), each with its own
+ * input rows, sign vectors, weights and shape, e.g. the seven matrices of one
+ * transformer layer (q, k, v, o, gate, up, down) in a verify sweep where each
+ * has its own activation rows.  The orcasaq2-rocm README (opening
+ * paragraph) cuts the launches of a decode step by fusing steps; here the
+ * same idea is applied to a layer's products: the whole group's work is split
+ * over the GPU as one problem, so the small matrices leave no SMs idle, and
+ * one launch (m = 1) or two (m >= 2: one rotation pre-pass for every member,
+ * then one product launch) serve the group.
+ *   m      : 1..32 rows, the same for every member.
+ *   probs  : HOST array of n_probs (1..8) exl3_problem_t, each with device
+ *            pointers x (m x k_in fp16), su (k_in), packed, scale (n_out), sv
+ *            (n_out) and y (m x n_out, fp16 or fp32 as y_fp32), and its k_in
+ *            and n_out (positive multiples of 128).  All members have `bits`
+ *            bits per weight.
+ *   workspace, ws_bytes : at least exl3_grouped_workspace_bytes(m, probs,
+ *            n_probs, bits) bytes, 256-byte aligned, zero-filled before first
+ *            use; reusable by later calls on the same stream.
+ * Each y_i equals the separate product's within rounding (the work split
+ * differs); repeated calls are bitwise identical.  The size query reads
+ * only k_in and n_out of each problem (the pointers may be NULL there) and
+ * returns 0 for an invalid group.
+ */
+typedef struct exl3_problem {
+    const uint16_t *x;
+    const uint16_t *su;
+    const uint32_t *packed;
+    const uint16_t *scale;
+    const uint16_t *sv;
+    void *y;
+    int k_in;
+    int n_out;
+} exl3_problem_t;
+
+EXL3_API size_t exl3_grouped_workspace_bytes(int m, const exl3_problem_t *probs, int n_probs, int bits);
+EXL3_API int exl3_gemm_grouped(int m, const exl3_problem_t *probs, int n_probs, int y_fp32, int bits,
+                               void *workspace, size_t ws_bytes, void *stream);
 
 /*
  * exl3_gemv_noalloc -- exl3_gemv without a workspace argument.  The source
