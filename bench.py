@@ -50,6 +50,8 @@ def parse():
                     help="input rows; above 32 the products go through the many-row (prefill) call, "
                          "with the synthetic rows repeated to m")
     ap.add_argument("--layers", type=int, default=64)
+    ap.add_argument("--first-layer", type=int, default=0,
+                    help="start the stack at this layer (e.g. a 2-bit layer for a profile capture)")
     ap.add_argument("--separate", action="store_true", help="one library call per matrix instead of per layer")
     ap.add_argument("--no-graph", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="time only the main row count (no M=1/8/16, no chain)")
@@ -268,9 +270,9 @@ def run_reference(args, world, rank):
 
 # ------------------------------------------------------------------ ours ----
 
-def make_weights(torch, device, layers, only=None):
+def make_weights(torch, device, layers, only=None, first=0):
     """Packed trellis words of the stack, generated on the device (SplitMix64)."""
-    specs = [s for s in synth.workload(5, m=32) if s.layer < layers]
+    specs = [s for s in synth.workload(5, m=32) if first <= s.layer < first + layers]
     if only:
         specs = [s for s in specs if s.name.split(".")[1] == only]
     return specs, [synth.splitmix64_words_torch(s.stream_id, s.n_words, device) for s in specs]
@@ -312,7 +314,7 @@ def run_ours(args, world, rank, local):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
-    specs, weights = make_weights(torch, device, args.layers, args.only)
+    specs, weights = make_weights(torch, device, args.layers, args.only, args.first_layer)
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
     full_layers = args.only is None
     extra = not args.no_extra and args.m <= 32

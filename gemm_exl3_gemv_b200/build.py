@@ -30,24 +30,36 @@ def _inputs():
         [os.path.join(ROOT, "include", "exl3.h")]
 
 
-def stale() -> bool:
-    if not os.path.exists(LIB):
+# The debug-bounds variant: every product kernel checks the index of each
+# access to the packed words, the workspace and the outputs, records a failed
+# check in the workspace status word and skips the access (no trap).
+LIB_DEBUG = os.path.join(HERE, "libexl3_debug.so")
+
+
+def stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return any(os.path.getmtime(p) > t for p in _inputs())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not stale():
-        return LIB
+def _compile(lib: str, extra, verbose: bool):
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc, *ARCH, *FLAGS, "-shared", "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc, *ARCH, *FLAGS, *extra, "-shared", "-I", os.path.join(ROOT, "include"), "-o", tmp, *sources()]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd))
     subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool = True) -> str:
+    """Build libexl3.so (and, unless debug=False, libexl3_debug.so) if stale."""
+    if force or stale(LIB):
+        _compile(LIB, [], verbose)
+    if debug and (force or stale(LIB_DEBUG)):
+        _compile(LIB_DEBUG, ["-DEXL3_DEBUG_BOUNDS"], verbose)
     return LIB
 
 

@@ -42,7 +42,8 @@ int validate_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16
 {
     if (!x || !packed || !scale || !su || !sv || !y) return EXL3_ERR_INVALID_ARG;
     if (m <= 0 || k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
-    if (m > 32 || !bits_ok(bits) || k_in % 128 || n_out % 128) return EXL3_ERR_UNSUPPORTED;
+    if (m > 32 || !bits_ok(bits) || k_in % 128 || n_out % 128 || n_out / 128 > exl3::kMaxBlocks)
+        return EXL3_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(su) || !aligned16(sv) ||
         !aligned16(y))
         return EXL3_ERR_MISALIGNED;
@@ -54,7 +55,7 @@ int validate_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16
 // Problem description of a single product (a group of one member).
 exl3::GemmArgs single_args(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* scale,
                            const uint16_t* su, const uint16_t* sv, void* y, int y_fp32, int k_in, int n_out,
-                           int bits, void* ws)
+                           int bits, void* ws, size_t ws_bytes)
 {
     exl3::GemmArgs a = {};
     a.y_fp32 = y_fp32 ? 1 : 0;
@@ -65,6 +66,7 @@ exl3::GemmArgs single_args(int m, const uint16_t* x, const uint32_t* packed, con
     a.mem[0] = exl3::Member{x, su, packed, scale, sv, y, k_in, n_out, 0, 0, 0, 0};
     exl3::finish_group(a);
     a.ws = static_cast<unsigned char*>(ws);
+    a.ws_bytes = ws_bytes;
     a.pdl = 1;
     return a;
 }
@@ -82,7 +84,7 @@ int run_gemm(int m, const uint16_t* x, const uint32_t* packed, const uint16_t* s
     if (st != EXL3_OK) return st;
     st = check_arch();
     if (st != EXL3_OK) return st;
-    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws);
+    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws, ws_bytes);
     cudaError_t e = launch_product(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }
@@ -102,6 +104,7 @@ const char* exl3_status_string(int status)
         case EXL3_ERR_ARCH: return "EXL3_ERR_ARCH: current device is not a compute capability 10.0 GPU";
         case EXL3_ERR_CUDA: return "EXL3_ERR_CUDA: a CUDA runtime call failed (see exl3_last_cuda_error)";
         case EXL3_ERR_TIMEOUT: return "EXL3_ERR_TIMEOUT: a kernel gave up a bounded wait; output invalid";
+        case EXL3_ERR_BOUNDS: return "EXL3_ERR_BOUNDS: a debug-build index check failed; output invalid";
     }
     return "EXL3: unknown status";
 }
@@ -112,13 +115,17 @@ int exl3_version(void) { return 100; }
 
 size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits)
 {
-    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
+    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits) ||
+        n_out / 128 > exl3::kMaxBlocks)
+        return 0;
     return m == 1 ? exl3::m1_workspace_bytes(k_in, n_out, bits) : exl3::tc_workspace_bytes(m, k_in, n_out, bits);
 }
 
 int exl3_kernel_launches(int m, int k_in, int n_out, int bits)
 {
-    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits)) return 0;
+    if (m <= 0 || m > 32 || k_in <= 0 || n_out <= 0 || k_in % 128 || n_out % 128 || !bits_ok(bits) ||
+        n_out / 128 > exl3::kMaxBlocks)
+        return 0;
     return m == 1 ? 1 : 2;
 }
 
@@ -136,7 +143,7 @@ int exl3_workspace_status(void* workspace, void* stream)
     if (e != cudaSuccess) return cuda_fail(e);
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e);
-    return EXL3_ERR_TIMEOUT;
+    return (word & exl3::kStatusBounds) ? EXL3_ERR_BOUNDS : EXL3_ERR_TIMEOUT;
 }
 
 int exl3_decode_tiles(const uint32_t* packed, int k_in, int n_out, int bits, uint16_t* w_out, void* stream)
@@ -200,7 +207,7 @@ extern "C" int exl3_gemm_large_m(int m, const uint16_t* x, const uint32_t* packe
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
     int st = check_arch();
     if (st != EXL3_OK) return st;
-    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, workspace);
+    exl3::GemmArgs a = single_args(m, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, workspace, ws_bytes);
     cudaError_t e = exl3::launch_gemm_large(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }
@@ -227,7 +234,7 @@ extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, 
         a.mem[i] = exl3::Member{x, su, t.packed, t.scale, t.sv, t.y, k_in, t.n_out, 0, 0, 0, 0};
         total += t.n_out;
     }
-    if (total > (1LL << 30)) return EXL3_ERR_UNSUPPORTED;
+    if (total / 128 > exl3::kMaxBlocks) return EXL3_ERR_UNSUPPORTED;
     const int n_total = (int)total;
     if (!workspace || ws_bytes < exl3_workspace_bytes(m, k_in, n_total, bits)) return EXL3_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return EXL3_ERR_MISALIGNED;
@@ -240,6 +247,7 @@ extern "C" int exl3_gemm_siblings(int m, const uint16_t* x, const uint16_t* su, 
     a.shared_x = 1;
     exl3::finish_group(a);
     a.ws = static_cast<unsigned char*>(workspace);
+    a.ws_bytes = ws_bytes;
     a.pdl = 1;
     cudaError_t e = launch_product(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
@@ -269,7 +277,7 @@ int grouped_args(int m, const exl3_problem_t* probs, int n_probs, int y_fp32, in
         a.mem[i] = exl3::Member{t.x, t.su, t.packed, t.scale, t.sv, t.y, t.k_in, t.n_out, 0, 0, 0, 0};
         total += t.n_out;
     }
-    if (total > (1LL << 30)) return EXL3_ERR_UNSUPPORTED;
+    if (total / 128 > exl3::kMaxBlocks) return EXL3_ERR_UNSUPPORTED;
     a.y_fp32 = y_fp32 ? 1 : 0;
     a.m = m;
     a.bits = bits;
@@ -305,6 +313,7 @@ extern "C" int exl3_gemm_grouped(int m, const exl3_problem_t* probs, int n_probs
     st = check_arch();
     if (st != EXL3_OK) return st;
     a.ws = static_cast<unsigned char*>(workspace);
+    a.ws_bytes = ws_bytes;
     cudaError_t e = launch_product(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);
 }
@@ -355,7 +364,7 @@ extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, cons
 {
     if (!x || !packed || !scale || !su || !sv || !y) return EXL3_ERR_INVALID_ARG;
     if (k_in <= 0 || n_out <= 0) return EXL3_ERR_INVALID_ARG;
-    if (!bits_ok(bits) || k_in % 128 || n_out % 128) return EXL3_ERR_UNSUPPORTED;
+    if (!bits_ok(bits) || k_in % 128 || n_out % 128 || n_out / 128 > exl3::kMaxBlocks) return EXL3_ERR_UNSUPPORTED;
     if (!aligned16(x) || !aligned16(packed) || !aligned16(scale) || !aligned16(su) || !aligned16(sv) ||
         !aligned16(y))
         return EXL3_ERR_MISALIGNED;
@@ -369,9 +378,9 @@ extern "C" int exl3_gemv_noalloc(const uint16_t* x, const uint32_t* packed, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     // the array keeps the last call's contents: the status word and the
     // arrival counters must start at zero
-    cudaError_t e = cudaMemsetAsync(ws, 0, exl3::ws_part_off(n_out), s);
+    cudaError_t e = cudaMemsetAsync(ws, 0, exl3::ws_data_off(), s);
     if (e != cudaSuccess) return cuda_fail(e);
-    exl3::GemmArgs a = single_args(1, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws);
+    exl3::GemmArgs a = single_args(1, x, packed, scale, su, sv, y, y_fp32, k_in, n_out, bits, ws, kNoAllocScratchBytes);
     a.pdl = 0;                       // follows a memset: ordinary stream order
     e = exl3::launch_gemv_m1(a, s);
     return e == cudaSuccess ? EXL3_OK : cuda_fail(e);

@@ -16,15 +16,46 @@ namespace exl3 {
 //                     its first v - 1 copies of the rotated input, so the wait
 //                     for the next one runs out (zero in normal use: the
 //                     workspace is zero-filled)
-// [256, 256 + 4*G)    one arrival counter per 128-channel output block
-// [ws_part_off, ...)  split-K partial sums, fp32 [splits][m][n_out]
+// [256, 256 + 4*kMaxBlocks)  one arrival counter per 128-channel output block;
+//                     a FIXED region, so that no call's partial sums or rotated
+//                     input ever land on another call's counters when calls of
+//                     different widths share a workspace (every call leaves the
+//                     counters it used at zero)
+// [ws_data_off(), ...) the call's own data: split-K partial sums, rotated input
 constexpr size_t kWsHeader = 256;
 constexpr uint32_t kStatusTimeout = 1u;
+constexpr uint32_t kStatusBounds = 2u;     // debug builds: an index check failed
 constexpr size_t kWsInjectOff = 4;
 
+// Debug builds (compiled with -DEXL3_DEBUG_BOUNDS): the kernels check the
+// index of every global access to the packed words, the workspace and the
+// outputs against the size of the array it touches.  guard(ok, status)
+// returns ok; a failed check also records kStatusBounds in the workspace
+// status word, and the caller skips the access (a load gives zeros) -- never a
+// trap, so the context stays usable.  Release builds compile the checks away.
+#ifdef EXL3_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+#ifdef __CUDACC__
+__device__ __forceinline__ bool guard(bool ok, uint32_t* status)
+{
+    if constexpr (kDebugBounds) {
+        if (!ok) atomicOr(status, kStatusBounds);
+        return ok;
+    } else {
+        return true;
+    }
+}
+#endif
+
 __host__ __device__ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+// output blocks (128 channels) of one call, summed over a group: at most
+// kMaxBlocks (1,048,576 output channels)
+constexpr int kMaxBlocks = 8192;
 __host__ __device__ inline size_t ws_counter_off() { return kWsHeader; }
-__host__ __device__ inline size_t ws_part_off(int n_out) { return align_up(kWsHeader + 4 * (size_t)(n_out / 128), 256); }
+__host__ __device__ inline size_t ws_data_off() { return align_up(kWsHeader + 4 * (size_t)kMaxBlocks, 256); }
 
 // ------------------------------------------------------------ addressing ---
 __device__ __forceinline__ uint32_t smem_u32(const void* p)

@@ -176,4 +176,18 @@ __device__ __forceinline__ void load_lane_words(uint32_t (&w)[2 * BITS], const u
     }
 }
 
+// load_lane_words, or zeros when the debug bounds check (the lane's words
+// inside the matrix's n_words) fails.
+template <int BITS>
+__device__ __forceinline__ void load_lane_words_checked(uint32_t (&w)[2 * BITS], const uint32_t* src,
+                                                        const uint32_t* base, size_t n_words, uint32_t* status)
+{
+    if (guard(src >= base && (size_t)(src - base) + 2 * BITS <= n_words, status)) {
+        load_lane_words<BITS>(w, src);
+    } else {
+#pragma unroll
+        for (int t = 0; t < 2 * BITS; ++t) w[t] = 0u;
+    }
+}
+
 }  // namespace exl3

@@ -46,6 +46,7 @@ struct GemmArgs {
     int shared_x;             // every member takes the same x and su (sibling group)
     Member mem[kMaxMembers];
     unsigned char* ws;        // workspace base
+    size_t ws_bytes;          // workspace size (checked by the debug-bounds build)
     int pdl;                  // launch with programmatic dependent launch (overlap the previous kernel's tail)
 };
 

@@ -45,7 +45,8 @@ constexpr uint64_t kLgWaitNs = 2000000000ull;
 // ------------------------------------------------------------- 1. decode ---
 template <int BITS>
 __global__ void __launch_bounds__(256) decode_aimage_kernel(const uint32_t* __restrict__ packed, int k_in, int n_out,
-                                                            uint8_t* __restrict__ image, uint32_t two16)
+                                                            uint8_t* __restrict__ image, uint32_t two16,
+                                                            uint32_t* status)
 {
     constexpr int TW = 8 * BITS, QW = 2 * BITS;
     grid_dep_wait();                                  // the image is read by the previous call's GEMM
@@ -55,7 +56,8 @@ __global__ void __launch_bounds__(256) decode_aimage_kernel(const uint32_t* __re
     if (item >= (long long)(n_out / 128) * T) return;
     const int g = (int)(item / T), tr = (int)(item % T);
     uint32_t w[QW];
-    load_lane_words<BITS>(w, packed + ((size_t)tr * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW);
+    load_lane_words_checked<BITS>(w, packed + ((size_t)tr * tiles_n + 8 * (size_t)g) * TW + (size_t)lane * QW, packed,
+                                  (size_t)T * tiles_n * TW, status);
     const int q = lane & 3;
     uint32_t buf[QW + 1];
     buf[0] = __shfl_sync(0xffffffffu, w[QW - 1], (lane & ~3) | ((q + 3) & 3));
@@ -64,8 +66,9 @@ __global__ void __launch_bounds__(256) decode_aimage_kernel(const uint32_t* __re
     uint32_t soff[2][2];
     lane_soff(lane, soff);
     uint8_t* dst = image + ((size_t)g * T + tr) * 4096;
+    const bool in = guard(((size_t)g * T + tr + 1) * 4096 <= (size_t)k_in * n_out * 2, status);
     decode_quarter_to_a<BITS>(buf, soff, two16, [&](uint32_t off, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3) {
-        *reinterpret_cast<uint4*>(dst + off) = make_uint4(w0, w1, w2, w3);
+        if (in) *reinterpret_cast<uint4*>(dst + off) = make_uint4(w0, w1, w2, w3);
     });
     grid_dep_launch();
 }
@@ -203,6 +206,12 @@ __global__ void __launch_bounds__(kLgThreads, 1) gemm_large_kernel(LgParams prm)
             tile_of(prm, G, t, g, j);
             const uint8_t* a_src = prm.image + (size_t)g * C64 * kAChunk;
             const uint8_t* b_src = prm.xt + (size_t)j * C64 * L::BCHUNK;
+            if (!guard((size_t)(g + 1) * C64 * kAChunk <= (size_t)prm.k_in * prm.n_out * 2 &&
+                           (size_t)(j + 1) * C64 * L::BCHUNK <= (size_t)prm.J * NB * prm.k_in * 2,
+                       prm.status)) {
+                ok = false;
+                break;
+            }
             for (int c = 0; c < C64; ++c, ++q) {
                 const int s = q % L::STAGES;
                 if (q >= L::STAGES && !lg_wait(&empty[s], (uint32_t)(q / L::STAGES - 1) & 1u, abort_flag)) {
@@ -390,7 +399,7 @@ cudaError_t launch_gemm_large_nb(const LgParams& prm, cudaStream_t stream, int p
 
 template <int BITS>
 cudaError_t launch_decode_image(const uint32_t* packed, int k_in, int n_out, uint8_t* image, cudaStream_t stream,
-                                int pdl)
+                                int pdl, uint32_t* status)
 {
     const long long items = (long long)(n_out / 128) * (k_in / 16);
     cudaLaunchConfig_t cfg = {};
@@ -402,7 +411,7 @@ cudaError_t launch_decode_image(const uint32_t* packed, int k_in, int n_out, uin
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, decode_aimage_kernel<BITS>, packed, k_in, n_out, image, 0x10000u);
+    return cudaLaunchKernelEx(&cfg, decode_aimage_kernel<BITS>, packed, k_in, n_out, image, 0x10000u, status);
 }
 
 }  // namespace
@@ -418,9 +427,9 @@ cudaError_t launch_gemm_large(const GemmArgs& a, cudaStream_t stream)
 
     cudaError_t e = cudaErrorInvalidValue;
     switch (a.bits) {
-        case 2: e = launch_decode_image<2>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
-        case 3: e = launch_decode_image<3>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
-        case 4: e = launch_decode_image<4>(sb.packed, k_in, a.n_out, image, stream, a.pdl); break;
+        case 2: e = launch_decode_image<2>(sb.packed, k_in, a.n_out, image, stream, a.pdl, reinterpret_cast<uint32_t*>(a.ws)); break;
+        case 3: e = launch_decode_image<3>(sb.packed, k_in, a.n_out, image, stream, a.pdl, reinterpret_cast<uint32_t*>(a.ws)); break;
+        case 4: e = launch_decode_image<4>(sb.packed, k_in, a.n_out, image, stream, a.pdl, reinterpret_cast<uint32_t*>(a.ws)); break;
     }
     if (e != cudaSuccess) return e;
     {

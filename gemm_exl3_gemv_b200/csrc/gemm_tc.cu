@@ -104,6 +104,8 @@ struct TcParams {
     float* part;            // stream-K partial sums, [slot][NT][128]
     uint32_t* counters;     // stream-K arrival counters, per output block
     uint32_t* status;       // workspace status word
+    size_t xt_bytes;        // size of the rotated-input region (debug-bounds checks)
+    int nslots;             // partial-sum slots in the workspace (debug-bounds checks)
     int S;                  // cluster size (CTAs per output block), 0: stream-K
     int P;                  // stream-K CTAs
     long long U;            // units: sum over members of blocks x 128-row input blocks
@@ -185,6 +187,8 @@ __device__ __forceinline__ void finish_row_regs(const GemmArgs& a, int g, int mm
 {
     const MemView sib = member_of_block(a, g);            // the matrix holding block g
     const int n0 = 128 * sib.gl + 4 * lane;
+    // warp-uniform (the rotation below shuffles across the warp)
+    if (!guard(mm < a.m && 128 * sib.gl + 128 <= sib.n_out, reinterpret_cast<uint32_t*>(a.ws))) return;
     const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
     const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
     const float2 sc0 = __half22float2(*reinterpret_cast<const __half2*>(&sc.x));
@@ -283,6 +287,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 if (kk >= kBStages && !wait_or_abort(&bempty[s], (uint32_t)(kk / kBStages - 1) & 1u, abort_flag)) break;
                 const MemView um = member_of_unit(a, u);
                 const int c = (int)((u - um.u0) % (um.k_in / 128));
+                if (!guard(um.xt0 + (size_t)(c + 1) * L::BUNIT <= prm.xt_bytes, prm.status)) break;
                 mbar_arrive_expect_tx(&bfull[s], L::BUNIT);
                 bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + um.xt0 + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
             }
@@ -328,6 +333,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             const uint32_t* src =
                 sib.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
             const size_t unit_step = (size_t)8 * tiles_n * TW;    // words between consecutive units
+            const size_t n_words = (size_t)C * 8 * tiles_n * TW;
             bool ok = true;                                      // warp-uniform
             // decode the segment's unit k (the CTA's kk-th) from `wds` into A
             // stage kk & 1, then lane 0 issues its MMA into this warp's accumulator
@@ -365,13 +371,14 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 }
             };
             uint32_t wa[QW], wb[QW];
-            load_lane_words<BITS>(wa, src);
+            load_lane_words_checked<BITS>(wa, src, sib.packed, n_words, prm.status);
             if (seg == 0) grid_dep_wait();     // weights are never written; y and the workspace after this
             int k = 0;
             for (; k + 2 <= nseg; k += 2) {
-                load_lane_words<BITS>(wb, src + (size_t)(k + 1) * unit_step);
+                load_lane_words_checked<BITS>(wb, src + (size_t)(k + 1) * unit_step, sib.packed, n_words, prm.status);
                 unit(wa, k, kk + k);
-                if (k + 2 < nseg) load_lane_words<BITS>(wa, src + (size_t)(k + 2) * unit_step);
+                if (k + 2 < nseg)
+                    load_lane_words_checked<BITS>(wa, src + (size_t)(k + 2) * unit_step, sib.packed, n_words, prm.status);
                 unit(wb, k + 1, kk + k + 1);
             }
             if (k < nseg) unit(wa, k, kk + k);
@@ -417,7 +424,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 const int p_last = cta_of_unit(ublk + C - 1, prm.P, prm.U);
                 float4* myslot = reinterpret_cast<float4*>(prm.part + (size_t)(p + g) * NT * 128);
                 const float4* z4s = reinterpret_cast<const float4*>(zsm);
-                for (int f = threadIdx.x; f < a.m * 32; f += 32 * kDec) __stcg(myslot + f, z4s[f]);
+                if (guard(p + g < prm.nslots, prm.status))
+                    for (int f = threadIdx.x; f < a.m * 32; f += 32 * kDec) __stcg(myslot + f, z4s[f]);
                 __threadfence();
                 named_bar(1, 32 * kDec);
                 if (threadIdx.x == 0) {
@@ -428,7 +436,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 finish = misc[2] != 0;
                 if (finish) {
                     __threadfence();
-                    reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, threadIdx.x, zsm);
+                    if (guard(p_first + g >= 0 && p_last + g < prm.nslots, prm.status))
+                        reduce_segments<NT>(prm.part, g, p_first, p_last, a.m, threadIdx.x, zsm);
                     if (threadIdx.x == 0) prm.counters[g] = 0u;      // ready for the next call on this stream
                     named_bar(1, 32 * kDec);
                 }
@@ -494,7 +503,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
 // placed at position 8(r >> 1) + 4(r & 1) + q.  One warp item = (member,
 // row, 128-block); a sibling group (shared x) rotates member 0's x only.
 template <int NT>
-__global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8_t* __restrict__ xt_base)
+__global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8_t* __restrict__ xt_base,
+                                                         size_t xt_bytes)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     grid_dep_launch();                 // the product kernel may start its prologue
@@ -525,7 +535,6 @@ __global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8
     if (!found) return;
     const int nblk = k_in / 128;
     const int m = (int)(item / nblk), b = (int)(item % nblk);
-    uint8_t* xt = const_cast<uint8_t*>(xt_base) + xt0;
     // lane holds elements i = (lane & 3) | (e << 2) | ((lane >> 2) << 4)
     float v[4];
 #pragma unroll
@@ -537,7 +546,10 @@ __global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8
     const int tr = 8 * b + (lane >> 2);
     const int pk0 = 16 * tr + 8 * ((lane >> 1) & 1) + 4 * (lane & 1);
     const int kchunk = pk0 >> 6, o = pk0 & 63, c16 = o >> 3, pos = o & 7;
-    uint8_t* dst = xt + (size_t)kchunk * NT * 128 + (m >> 3) * 1024 + (m & 7) * 128 + ((c16 ^ (m & 7)) << 4) + pos * 2;
+    const size_t doff = (size_t)xt0 + (size_t)kchunk * NT * 128 + (m >> 3) * 1024 + (m & 7) * 128 +
+                        ((c16 ^ (m & 7)) << 4) + pos * 2;
+    if (!guard(doff + 8 <= xt_bytes, reinterpret_cast<uint32_t*>(a.ws))) return;
+    uint8_t* dst = const_cast<uint8_t*>(xt_base) + doff;
     __half2 h2[2] = {__floats2half2_rn(v[0] * kInvSqrt128, v[1] * kInvSqrt128),
                      __floats2half2_rn(v[2] * kInvSqrt128, v[3] * kInvSqrt128)};
     *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<uint2*>(h2);
@@ -545,7 +557,7 @@ __global__ void __launch_bounds__(256) xt_prepass_kernel(GemmArgs a, const uint8
 
 int nt_for(int m) { return m <= 16 ? 16 : 32; }
 
-size_t xt_offset(int G) { return align_up(ws_counter_off() + 4 * (size_t)G, 1024); }
+size_t xt_offset(int G) { (void)G; return align_up(ws_data_off(), 1024); }
 
 // Units of the group (sum over members of blocks x 128-row input blocks).
 long long group_units(const GemmArgs& a)
@@ -692,6 +704,8 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
     const size_t xt_off = xt_offset(G);
     prm.xt = ws + xt_off;
     prm.part = reinterpret_cast<float*>(ws + part_offset(a, NT));
+    prm.xt_bytes = xt_bytes(a, NT);
+    prm.nslots = sk_ctas(G, prm.U) + G;
 
     long long items = 0;
     for (int i = 0; i < (a.shared_x ? 1 : a.nmem); ++i) items += (long long)NT * (a.mem[i].k_in / 128);
@@ -705,7 +719,8 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
         pcfg.stream = stream;
         pcfg.attrs = &pdl_attr;
         pcfg.numAttrs = a.pdl ? 1 : 0;
-        cudaError_t e = cudaLaunchKernelEx(&pcfg, xt_prepass_kernel<NT>, a, (const uint8_t*)(ws + xt_off));
+        cudaError_t e = cudaLaunchKernelEx(&pcfg, xt_prepass_kernel<NT>, a, (const uint8_t*)(ws + xt_off),
+                                           xt_bytes(a, NT));
         if (e != cudaSuccess) return e;
     }
     cudaError_t e = cudaGetLastError();

@@ -141,42 +141,58 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     const long long b0 = (long long)p * pl.U / pl.P, b1 = (long long)(p + 1) * pl.U / pl.P;
     const int q = lane & 3;
     const int src_prev = (lane & ~3) | ((q + 3) & 3);
-    float* part = reinterpret_cast<float*>(a.ws + ws_part_off(a.n_out));
+    float* part = reinterpret_cast<float*>(a.ws + ws_data_off());
     uint32_t* counters = reinterpret_cast<uint32_t*>(a.ws + ws_counter_off());
+    uint32_t* status = reinterpret_cast<uint32_t*>(a.ws);
+    const int G = a.n_out / 128;
+    // partial slot s is in bounds (debug builds)
+    auto slot_ok = [&](long long s) {
+        return guard(s >= 0 && s < (long long)pl.P + G &&
+                         ws_data_off() + (size_t)(s + 1) * 128 * sizeof(float) <= a.ws_bytes,
+                     status);
+    };
     grid_dep_launch();                     // the next product may start loading its weights
     bool first_seg = true;
 
     for (long long u = b0; u < b1;) {
-        // ---- segment: block g (group numbering) = block gl of member mv, tile rows [r0, r1) ----
-        const MemView mv = member_of_unit(a, u);
-        const int T = mv.k_in / 16;                                    // tile rows per block of this member
-        const int gl = (int)((u - mv.u0) / T);
-        const int g = mv.g0 + gl;
-        const long long ublk = mv.u0 + (long long)gl * T;              // the block's first unit
-        const int r0 = (int)(u - ublk);
-        const int r1 = (int)((ublk + T < b1 ? ublk + T : b1) - ublk);
+        // ---- segment: block g (group numbering), tile rows [r0, r1) of its member ----
+        // (the member view is looked up again after the main loop, from g, so
+        // that nothing of it stays live in registers across the decode)
+        int g, r0, r1;
+        const uint32_t* src;
+        const uint32_t* wbase;                                         // the member's packed words
+        size_t row_step, n_words;                                      // words between a warp's rows; matrix size
+        {
+            const MemView mv = member_of_unit(a, u);
+            const int T = mv.k_in / 16;                                // tile rows per block of this member
+            const int gl = (int)((u - mv.u0) / T);
+            g = mv.g0 + gl;
+            const long long ublk = mv.u0 + (long long)gl * T;          // the block's first unit
+            r0 = (int)(u - ublk);
+            r1 = (int)((ublk + T < b1 ? ublk + T : b1) - ublk);
+            const int tiles_n = mv.n_out / 16;
+            row_step = (size_t)kM1Warps * tiles_n * TW;
+            n_words = (size_t)T * tiles_n * TW;
+            wbase = mv.packed;
+            src = mv.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
+        }
         u += r1 - r0;
         const int kb_lo = r0 >> 3, kb_hi = (r1 + 7) >> 3;             // 128-row input blocks touched
         const int nrow = r1 - r0;
         const int nw = nrow > warp ? (nrow - warp + kM1Warps - 1) / kM1Warps : 0;
-        size_t row_step;                                               // words between a warp's rows
-        const uint32_t* src;
-        {
-            const int tiles_n = mv.n_out / 16;
-            row_step = (size_t)kM1Warps * tiles_n * TW;
-            src = mv.packed + ((size_t)(r0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
-        }
         uint32_t wa[QW], wb[QW];
-        if (nw > 0) load_lane_words<BITS>(wa, src);                       // in flight during the rotation
+        if (nw > 0) load_lane_words_checked<BITS>(wa, src, wbase, n_words, status);   // in flight during the rotation
         if (first_seg) grid_dep_wait();    // weights are never written; x, y, workspace only after this
         first_seg = false;
 
         __syncthreads();                                               // previous segment done with smem
         // input rotation of the touched blocks: xxs[k - 128 kb_lo] = (xt, xt)
         for (int kb = kb_lo + warp; kb < kb_hi; kb += kM1Warps) {
+            const MemView mv = member_of_block(a, g);
             const int col = kb * 128 + 4 * lane;
-            const uint2 raw = *reinterpret_cast<const uint2*>(mv.x + col);
-            const uint2 sraw = *reinterpret_cast<const uint2*>(mv.su + col);
+            const bool in = guard(col + 4 <= mv.k_in && kb - kb_lo < pl.kb_max, status);
+            const uint2 raw = in ? *reinterpret_cast<const uint2*>(mv.x + col) : make_uint2(0u, 0u);
+            const uint2 sraw = in ? *reinterpret_cast<const uint2*>(mv.su + col) : make_uint2(0u, 0u);
             const float2 x0 = __half22float2(as_h2(raw.x)), x1 = __half22float2(as_h2(raw.y));
             const float2 s0 = __half22float2(as_h2(sraw.x)), s1 = __half22float2(as_h2(sraw.y));
             float v[4] = {x0.x * s0.x, x0.y * s0.y, x1.x * s1.x, x1.y * s1.y};
@@ -187,7 +203,7 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
             h = __float2half2_rn(v[1] * kInvSqrt128); o.y = *reinterpret_cast<uint32_t*>(&h);
             h = __float2half2_rn(v[2] * kInvSqrt128); o.z = *reinterpret_cast<uint32_t*>(&h);
             h = __float2half2_rn(v[3] * kInvSqrt128); o.w = *reinterpret_cast<uint32_t*>(&h);
-            *reinterpret_cast<uint4*>(xxs + (kb - kb_lo) * 128 + 4 * lane) = o;
+            if (in) *reinterpret_cast<uint4*>(xxs + (kb - kb_lo) * 128 + 4 * lane) = o;
         }
         __syncthreads();
 
@@ -201,9 +217,9 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         __half2 acc[16];
         int i = 0;
         for (; i + 2 <= nw; i += 2) {
-            load_lane_words<BITS>(wb, src + (size_t)(i + 1) * row_step);
+            load_lane_words_checked<BITS>(wb, src + (size_t)(i + 1) * row_step, wbase, n_words, status);
             tile_row<BITS, true, ALT_EVERY>(wa, xxs, kx0 + i * kx_step, src_prev, acc, two16);
-            if (i + 2 < nw) load_lane_words<BITS>(wa, src + (size_t)(i + 2) * row_step);
+            if (i + 2 < nw) load_lane_words_checked<BITS>(wa, src + (size_t)(i + 2) * row_step, wbase, n_words, status);
             tile_row<BITS, false, ALT_EVERY>(wb, xxs, kx0 + (i + 1) * kx_step, src_prev, acc, two16);
 #pragma unroll
             for (int c = 0; c < 16; ++c) accf[c] = add_pair_f32(accf[c], acc[c]);
@@ -236,10 +252,13 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         }
 
         // ---- a block split over several CTAs: the last to arrive finishes it ----
+        const MemView mv = member_of_block(a, g);
+        const int T = mv.k_in / 16;
+        const long long ublk = mv.u0 + (long long)mv.gl * T;
         if (nrow < T) {
             const int p_first = m1_cta_of_unit(ublk, pl.P, pl.U);
             const int p_last = m1_cta_of_unit(ublk + T - 1, pl.P, pl.U);
-            if (threadIdx.x < 128) __stcg(part + (size_t)(p + g) * 128 + threadIdx.x, z);
+            if (threadIdx.x < 128 && slot_ok(p + g)) __stcg(part + (size_t)(p + g) * 128 + threadIdx.x, z);
             __threadfence();
             __syncthreads();
             if (threadIdx.x == 0) {
@@ -260,11 +279,12 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
                 for (; qq + 14 <= p_last; qq += 16) {
                     float v[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] = __ldcg(pp + (size_t)(qq + 2 * e) * 128);
+                    for (int e = 0; e < 8; ++e)
+                        v[e] = slot_ok(qq + 2 * e + g) ? __ldcg(pp + (size_t)(qq + 2 * e) * 128) : 0.f;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) zz += v[e];
                 }
-                for (; qq <= p_last; qq += 2) zz += __ldcg(pp + (size_t)qq * 128);
+                for (; qq <= p_last; qq += 2) zz += slot_ok(qq + g) ? __ldcg(pp + (size_t)qq * 128) : 0.f;
                 red[threadIdx.x] = zz;
                 __syncthreads();
                 if (threadIdx.x < 128) z = red[threadIdx.x] + red[128 + threadIdx.x];
@@ -276,9 +296,9 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         __syncthreads();
 
         // ---- epilogue (warp 0): scale, output rotation, signs, store ----
-        if (warp == 0) {
+        if (warp == 0 && guard(128 * mv.gl + 128 <= mv.n_out, status)) {
             const MemView sib = mv;
-            const int n0 = 128 * gl + 4 * lane;
+            const int n0 = 128 * mv.gl + 4 * lane;
             const float4 z4 = *reinterpret_cast<const float4*>(red + 4 * lane);
             const uint2 sc = *reinterpret_cast<const uint2*>(sib.scale + n0);
             const uint2 sg = *reinterpret_cast<const uint2*>(sib.sv + n0);
@@ -382,7 +402,7 @@ size_t m1_group_workspace_bytes(const GemmArgs& a0)
 {
     GemmArgs a = a0;
     const M1Plan pl = m1_plan(a);
-    return ws_part_off(a.n_out) + (size_t)(pl.P + a.n_out / 128) * 128 * sizeof(float);
+    return ws_data_off() + (size_t)(pl.P + a.n_out / 128) * 128 * sizeof(float);
 }
 
 size_t m1_workspace_bytes(int k_in, int n_out, int bits)

@@ -14,7 +14,9 @@ from typing import Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libexl3.so")
+# EXL3_LIBRARY selects another build of the library, e.g. the debug-bounds
+# build libexl3_debug.so next to this file.
+LIB_PATH = os.environ.get("EXL3_LIBRARY") or os.path.join(_HERE, "libexl3.so")
 
 EXL3_OK = 0
 EXL3_ERR_INVALID_ARG = 1
@@ -24,6 +26,7 @@ EXL3_ERR_WORKSPACE = 4
 EXL3_ERR_ARCH = 5
 EXL3_ERR_CUDA = 6
 EXL3_ERR_TIMEOUT = 7
+EXL3_ERR_BOUNDS = 8
 
 # every entry point include/exl3.h declares
 EXPORTS = ("exl3_status_string", "exl3_last_cuda_error", "exl3_version", "exl3_workspace_bytes",

@@ -61,13 +61,16 @@ enum {
     EXL3_OK = 0,
     EXL3_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad mode     */
     EXL3_ERR_UNSUPPORTED = 2,  /* bits not in {2,3,4}; shape not a multiple of
-                                  128 (16 for decode); m outside [1, 32]        */
+                                  128 (16 for decode); m outside [1, 32]; more
+                                  than 1,048,576 output channels in one call    */
     EXL3_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned               */
     EXL3_ERR_WORKSPACE = 4,    /* workspace null or smaller than required        */
     EXL3_ERR_ARCH = 5,         /* current device is not compute capability 10.0 */
     EXL3_ERR_CUDA = 6,         /* a CUDA runtime call failed                     */
-    EXL3_ERR_TIMEOUT = 7       /* a kernel's bounded wait expired (see
+    EXL3_ERR_TIMEOUT = 7,      /* a kernel's bounded wait expired (see
                                   exl3_workspace_status)                         */
+    EXL3_ERR_BOUNDS = 8        /* debug builds only: an index check inside a
+                                  kernel failed (see exl3_workspace_status)      */
 };
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -81,13 +84,16 @@ EXL3_API int exl3_version(void);
 
 /*
  * exl3_workspace_bytes -- size of the caller-allocated workspace that
- * exl3_gemv / exl3_gemm_small_m need for this problem: split-K partial sums
- * (fp32, L2-resident in practice), one arrival counter per 128-channel output
- * block and a status word.  The workspace must be zero-filled once before its
- * first use; every call leaves its counters at zero again, so it can be
- * reused by later calls on the SAME stream without clearing.  Calls that may
- * run concurrently need separate workspaces.  Returns 0 for an unsupported
- * problem.  Host-only, no CUDA call.
+ * exl3_gemv / exl3_gemm_small_m need for this problem: a status word, a fixed
+ * 32 KB region of arrival counters (one per 128-channel output block; at most
+ * 8192 blocks, i.e. 1,048,576 output channels, per call), then the call's own
+ * split-K partial sums (fp32, L2-resident in practice) and rotated input.
+ * The workspace must be zero-filled once before its first use; every call
+ * leaves the counters at zero again and writes its own data only past the
+ * counter region, so one workspace (sized for the largest call) serves any
+ * sequence of calls of any shapes on the SAME stream without clearing.  Calls
+ * that may run concurrently need separate workspaces.  Returns 0 for an
+ * unsupported problem.  Host-only, no CUDA call.
  */
 EXL3_API size_t exl3_workspace_bytes(int m, int k_in, int n_out, int bits);
 
@@ -103,6 +109,11 @@ EXL3_API int exl3_kernel_launches(int m, int k_in, int n_out, int bits);
  * workspace status word.  Returns EXL3_OK, or EXL3_ERR_TIMEOUT if a kernel
  * that used this workspace gave up a bounded wait (its output is then not
  * valid).  Every wait in the multi-row kernels gives up after 2 s.
+ * Debug builds (the library compiled with -DEXL3_DEBUG_BOUNDS, built as
+ * libexl3_debug.so next to libexl3.so) check the index of every access of the
+ * product kernels to the packed words, the workspace and the outputs; a
+ * failed check skips the access (no trap) and this call then returns
+ * EXL3_ERR_BOUNDS.
  * Testing that path: while the uint32 at byte offset 4 of the workspace is
  * nonzero, exl3_gemm_small_m (m >= 2) and exl3_gemm_siblings (m >= 2) let
  * only the first v - 1 rotated-input copies of each CTA through (v = the

@@ -36,6 +36,43 @@ def test_every_declared_symbol_is_exported(ex):
     assert set(names) == set(ex.EXPORTS)
 
 
+def test_debug_bounds_build_exports_the_same_symbols(ex):
+    from gemm_exl3_gemv_b200 import build
+    dbg = ctypes.CDLL(build.LIB_DEBUG)
+    for n in declared_entry_points():
+        assert hasattr(dbg, n), n
+    dbg.exl3_status_string.restype = ctypes.c_char_p
+    assert b"EXL3_ERR_BOUNDS" in dbg.exl3_status_string(ex.EXL3_ERR_BOUNDS)
+
+
+def test_grouped_validation(ex):
+    P = ex.Problem
+    # size query: shapes only, pointers may be NULL
+    two = (P * 2)(P(None, None, None, None, None, None, 5120, 1024), P(None, None, None, None, None, None, 17408, 5120))
+    assert ex.lib.exl3_grouped_workspace_bytes(1, two, 2, 3) > 0
+    assert ex.lib.exl3_grouped_workspace_bytes(32, two, 2, 3) > ex.lib.exl3_grouped_workspace_bytes(1, two, 2, 3)
+    assert ex.lib.exl3_grouped_workspace_bytes(33, two, 2, 3) == 0
+    assert ex.lib.exl3_grouped_workspace_bytes(1, two, 9, 3) == 0
+    bad = (P * 1)(P(None, None, None, None, None, None, 130, 128))
+    assert ex.lib.exl3_grouped_workspace_bytes(1, bad, 1, 3) == 0
+    # the call itself: NULL pointers are rejected before anything runs
+    st = ex.lib.exl3_gemm_grouped(1, two, 2, 0, 3, None, 0, None)
+    assert st == ex.EXL3_ERR_INVALID_ARG
+    assert ex.lib.exl3_gemm_grouped(1, two, 0, 0, 3, None, 0, None) == ex.EXL3_ERR_INVALID_ARG
+    assert ex.lib.exl3_gemm_grouped(1, two, 2, 0, 5, None, 0, None) == ex.EXL3_ERR_UNSUPPORTED
+
+
+def test_grouped_workspace_covers_separate_products(ex):
+    """The grouped workspace holds at least the largest member's own needs."""
+    P = ex.Problem
+    shapes = [(5120, 5120), (5120, 1024), (5120, 1024), (5120, 5120), (5120, 17408), (5120, 17408), (17408, 5120)]
+    arr = (P * 7)(*[P(None, None, None, None, None, None, k, n) for k, n in shapes])
+    for m in (1, 8, 32):
+        g = ex.lib.exl3_grouped_workspace_bytes(m, arr, 7, 3)
+        assert g >= max(ex.workspace_bytes(m, k, n, 3) for k, n in shapes) // 2
+        assert g % 16 == 0
+
+
 def test_version_and_status_strings(ex):
     assert ex.lib.exl3_version() >= 100
     for st in range(8):

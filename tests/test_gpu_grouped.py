@@ -29,7 +29,8 @@ def _dev_problems(inps, fp32):
     probs = []
     for inp in inps:
         s = inp.spec
-        y = torch.full((s.m, s.n_out), float("nan"), dtype=torch.float32 if fp32 else torch.float16, device="cuda")
+        rows = inp.x.shape[0]
+        y = torch.full((rows, s.n_out), float("nan"), dtype=torch.float32 if fp32 else torch.float16, device="cuda")
         probs.append((to_dev(inp.x), to_dev(inp.packed), to_dev(inp.scale), to_dev(inp.su), to_dev(inp.sv), y))
     return probs
 

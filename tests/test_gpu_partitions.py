@@ -64,3 +64,25 @@ def test_partitions_repeatable_bitwise(ex, k, n, m):
     for _ in range(4):
         assert torch.equal(ex.gemm(*args, 3, workspace=ws), first)
     assert ex.workspace_status(ws) == ex.EXL3_OK
+
+
+@pytest.mark.parametrize("m", [1, 8, 32])
+def test_shared_workspace_across_widths(m):
+    """Calls of different output widths (and the grouped call) back to back on
+    one workspace, sized for the largest: every output equals the same call on
+    a fresh workspace, bit for bit.  (A call's partial sums or rotated input
+    must never land on another call's arrival counters.)"""
+    import torch
+    from gemm_exl3_gemv_b200 import exl3 as ex
+    shapes = [(5120, 1024), (5120, 17408), (17408, 5120), (5120, 1024), (256, 40960), (5120, 17408)]
+    specs = [synth.MatrixSpec(f"sw{i}", k, n, 2, m, seed=150, index=i) for i, (k, n) in enumerate(shapes)]
+    inps = [synth.make_inputs(s) for s in specs]
+    dev = [[to_dev(a) for a in (i.x, i.packed, i.scale, i.su, i.sv)] for i in inps]
+    fresh = [ex.gemm(*d, 2).clone() for d in dev]
+    ws = torch.zeros(max(ex.workspace_bytes(m, k, n, 2) for k, n in shapes), dtype=torch.uint8, device="cuda")
+    for rep in range(2):
+        outs = [ex.gemm(*d, 2, workspace=ws) .clone() for d in dev]
+        torch.cuda.synchronize()
+        for s, f, o in zip(specs, fresh, outs):
+            assert torch.equal(f, o), f"{s.name} m={m} pass {rep}"
+    assert ex.workspace_status(ws) == ex.EXL3_OK

@@ -45,11 +45,11 @@ def test_noalloc_matches_workspace_gemv_twice(idx):
 def test_noalloc_rejects_problem_beyond_scratch():
     import torch
     from gemm_exl3_gemv_b200 import exl3 as ex
-    # 2**21 output blocks: the arrival counters alone need 8 MiB, beyond the
-    # 4 MiB scratch.  The host check (the same workspace size, host-only) must
-    # hold before the call, which then returns before anything is enqueued,
-    # so small stand-in buffers are enough.
-    k, n, bits = 128, 1 << 28, 2
+    # 8192 output blocks (the most one call takes): the partial sums alone
+    # need more than the 4 MiB scratch.  The host check (the same workspace
+    # size, host-only) must hold before the call, which then returns before
+    # anything is enqueued, so small stand-in buffers are enough.
+    k, n, bits = 128, 1 << 20, 2
     assert ex.workspace_bytes(1, k, n, bits) > 4 << 20
     buf = torch.zeros(64, dtype=torch.float16, device="cuda")
     assert _noalloc(ex, buf, buf, buf, buf, buf, buf, k, n, bits) == ex.EXL3_ERR_WORKSPACE
