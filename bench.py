@@ -278,6 +278,17 @@ def make_weights(torch, device, layers, only=None, first=0):
     return specs, [synth.splitmix64_words_torch(s.stream_id, s.n_words, device) for s in specs]
 
 
+def max_over_ranks(torch, dist, v: float, device) -> float:
+    """The largest of every rank's v (all ranks get it); v itself on one rank.
+    Each rank's step time is its own CUDA-event measurement; the job's step
+    time is the slowest rank's."""
+    if dist is None:
+        return v
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def timed(torch, fn, steps, warmup, barrier):
     for _ in range(warmup):
         fn()
@@ -307,12 +318,8 @@ def run_ours(args, world, rank, local):
     from gemm_exl3_gemv_b200 import exl3 as ex
     from gemm_exl3_gemv_b200.stack import Stack
 
-    def max_over_ranks(v):
-        if not dist:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v):
+        return max_over_ranks(torch, dist, v, device)
 
     specs, weights = make_weights(torch, device, args.layers, args.only, args.first_layer)
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(local).uuid)
@@ -343,15 +350,15 @@ def run_ours(args, world, rank, local):
         if sampler:
             sampler.start()
             time.sleep(0.5)                             # let nvidia-smi start sampling
-        ms = max_over_ranks(timed(torch, fn, args.steps, args.warmup, barrier))
+        ms = rank_max(timed(torch, fn, args.steps, args.warmup, barrier))
         clocks = sampler.stop() if sampler else None
         res = {"ms": ms, "launch": launch, "clocks": clocks, "launches": st.launches()}
         if m == args.m:
             # end to end through the binding from pinned host buffers: graphed, then eager
             fe, ge, elaunch = graph_or_eager(st, st.run_e2e)
-            res["e2e_ms"] = max_over_ranks(timed(torch, fe, args.steps, max(1, args.warmup), barrier))
+            res["e2e_ms"] = rank_max(timed(torch, fe, args.steps, max(1, args.warmup), barrier))
             res["e2e_launch"] = elaunch
-            res["e2e_eager_ms"] = max_over_ranks(timed(torch, st.run_e2e, args.steps, max(1, args.warmup), barrier))
+            res["e2e_eager_ms"] = rank_max(timed(torch, st.run_e2e, args.steps, max(1, args.warmup), barrier))
             assert ex.workspace_status(st.ws) == ex.EXL3_OK
             assert torch.equal(st.y_pin, st.y_dev.cpu()), "end-to-end outputs differ from the device outputs"
             del ge
@@ -368,7 +375,7 @@ def run_ours(args, world, rank, local):
         for m in ([args.m, 1] if args.m != 1 else [1]):
             st = Stack(ex, torch, device, m, specs, weights, mode="chain")
             fn, g, launch = graph_or_eager(st, st.run)
-            chain[m] = max_over_ranks(timed(torch, fn, args.steps, args.warmup, barrier))
+            chain[m] = rank_max(timed(torch, fn, args.steps, args.warmup, barrier))
             assert ex.workspace_status(st.ws) == ex.EXL3_OK
             del g, st
 

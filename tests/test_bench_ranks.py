@@ -30,3 +30,36 @@ def test_reference_arm_two_ranks_one_line():
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["unit"] == "GB/s"
     assert d["cpu_baseline"]["kind"] == "oracle" and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def _rank_worker(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks(torch, dist, 1.5 + rank, "cpu")     # each rank's own step time
+        out.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    """The step time bench.py reports under torchrun is the slowest rank's:
+    bench.max_over_ranks (the all-reduce MAX the repo arm runs over NCCL)
+    on two gloo ranks on CPU."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    out = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_worker, args=(r, 2, port, out)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(out.get(timeout=10) for _ in range(2))
+    assert res == {0: 2.5, 1: 2.5}
