@@ -359,9 +359,10 @@ size_t m1_smem_bytes(const M1Plan& pl)
 
 // Form of the window isolation per bit width (measured on B200): 2 and 4
 // bits read byte-aligned windows from shifted words; 3 bits (windows at
-// every bit offset) puts every second non-aligned window on the FMA pipe.
+// every bit offset) puts every third non-aligned window on the FMA pipe
+// (every second: 2-4 % slower; every one: 15 % slower).
 #ifndef EXL3_M1_ALT3
-#define EXL3_M1_ALT3 2
+#define EXL3_M1_ALT3 3
 #endif
 #ifndef EXL3_M1_ALT24
 #define EXL3_M1_ALT24 (-1)

@@ -76,13 +76,36 @@ def _oracle_chain(oracle_mod, specs, m, layers):
     return out
 
 
+def _chain_depth(spec):
+    """Products on the dependency path ending at this one: layer l's sibling
+    call (q, k, v, gate, up) is product 2l + 1 of the chain, its o and down
+    are product 2l + 2."""
+    kind = spec.name.split(".")[1]
+    return 2 * spec.layer + (2 if kind in ("o", "down") else 1)
+
+
 @pytest.mark.parametrize("m", [1, 32])
 def test_graphed_chain_matches_composed_oracle(oracle_mod, m):
+    """Tolerance: each product meets the per-product bound (rel-L2 1e-3,
+    max-abs 1e-2) on its own inputs (the other tests).  In a chain the input
+    of product d is the library's fp16 output of product d - 1, which already
+    differs from the oracle's; the products are near norm-preserving (scales
+    divided by their average gain), so a relative input error passes through
+    at about its own size and the errors of the d products on the path add:
+    rel-L2 <= d * 1e-3 and max-abs <= d * 1e-2 at depth d."""
+    import gpu_helpers
     layers = 2
     st = _stack(m, layers, "chain", False)
     _replay(st)
     ref = _oracle_chain(oracle_mod, st.specs, m, layers)
     for p in st.products:
-        check_close(p.y.cpu().numpy(), ref[p.spec.name], f"chain {p.spec.name} m={m}")
+        d = _chain_depth(p.spec)
+        got = p.y.cpu().numpy().astype(np.float64)
+        r = ref[p.spec.name]
+        rel = np.linalg.norm(got - r) / np.linalg.norm(r)
+        mx = np.abs(got - r).max()
+        assert np.all(np.isfinite(got)), p.spec.name
+        assert rel <= d * gpu_helpers.REL_L2, f"chain {p.spec.name} m={m} depth {d}: rel-L2 {rel:.3e}"
+        assert mx <= d * gpu_helpers.MAX_ABS, f"chain {p.spec.name} m={m} depth {d}: max-abs {mx:.3e}"
     # the chain is carried: layer 1's input is layer 0's down output
     assert np.abs(ref["l1.down"]).max() > 0
