@@ -387,20 +387,32 @@ def run_ours(args, world, rank, local):
     algo_bytes = st.packed_bytes + st.io_bytes
     achieved = algo_bytes / (main["ms"] * 1e-3) / 1e9
     n_weights = sum(s.n_weights for s in st.specs)
-    kname = "gemv_m1_counters" if args.m == 1 else "gemm_tc_counters"
-    cnt, cnt_why = counters(kname) if args.m <= 32 else (None, "many-row path")
+    sm_mhz = (main["clocks"] or {}).get("sm_mhz") or 1965.0
+    # one launch of the dominant kernel = one library call of the step: a whole
+    # layer (grouped) or one matrix (separate calls)
+    per_launch = len(st.layers) if st.grouped else len(st.specs)
+
+    def issue_record(m, ms):
+        """Instruction-issue roofline: committed instructions per weight (ncu)
+        x weights/s against 4 issue slots x 148 SMs x the sampled clock x 32 lanes."""
+        c, why = counters("gemv_m1_counters" if m == 1 else "gemm_tc_counters")
+        if c is None or "thread_instructions_per_weight" not in c:
+            return {"bound": "alu-issue", "frac": None, "why": why}, c, why
+        ipw = float(c["thread_instructions_per_weight"])
+        wps = n_weights / (ms * 1e-3)
+        peak_ti = 4 * 148 * sm_mhz * 1e6 * 32
+        return ({"bound": "alu-issue", "instr_per_weight": ipw, "weights_per_s_T": round(wps / 1e12, 4),
+                 "achieved": round(ipw * wps / 1e12, 3), "peak": round(peak_ti / 1e12, 3),
+                 "unit": "T thread-instr/s", "frac": round(ipw * wps / peak_ti, 4), "sm_mhz": sm_mhz,
+                 "source": c.get("capture")}, c, None)
+
+    if args.m <= 32:
+        issue, cnt, cnt_why = issue_record(args.m, main["ms"])
+    else:
+        issue, cnt, cnt_why = {"bound": "alu-issue", "frac": None, "why": "many-row path"}, None, "many-row path"
     traffic = None
     if cnt is not None and "dram_bytes_per_packed_byte" in cnt:
-        traffic = round(cnt["dram_bytes_per_packed_byte"] * st.packed_bytes / len(st.specs))
-    sm_mhz = (main["clocks"] or {}).get("sm_mhz") or 1965.0
-    issue = None
-    if cnt is not None and "thread_instructions_per_weight" in cnt:
-        ipw = float(cnt["thread_instructions_per_weight"])
-        wps = n_weights / (main["ms"] * 1e-3)
-        peak_ti = 4 * 148 * sm_mhz * 1e6 * 32                 # 4 issue slots x 148 SMs x clock x 32 lanes
-        issue = {"bound": "alu-issue", "instr_per_weight": ipw, "weights_per_s": round(wps / 1e12, 4),
-                 "achieved": round(ipw * wps / 1e12, 3), "peak": round(peak_ti / 1e12, 3), "unit": "T thread-instr/s",
-                 "frac": round(ipw * wps / peak_ti, 4), "sm_mhz": sm_mhz, "source": cnt.get("capture")}
+        traffic = round(cnt["dram_bytes_per_packed_byte"] * st.packed_bytes / per_launch)
     line = {
         "metric": METRIC, "value": round(gbs * world, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(main["ms"], 4),
@@ -428,11 +440,13 @@ def run_ours(args, world, rank, local):
                      "peak_kind": peak_kind,
                      "kernel": ("verify product (rotation pre-pass + gemm_tc_kernel)" if args.m > 1 else
                                 "single-row product (gemv_m1_kernel)") +
-                               ": algorithmic bytes per step / CUDA-event step time",
-                     "algorithmic_bytes_per_product": round(algo_bytes / len(st.specs)),
+                               ": algorithmic bytes per step / CUDA-event step time; one launch = " +
+                               ("one grouped layer call" if st.grouped else "one matrix"),
+                     "algorithmic_bytes_per_launch": round(algo_bytes / per_launch),
+                     "traffic_per": "launch (measured DRAM bytes per packed byte x the launch's packed bytes)",
                      "traffic_source": cnt.get("capture") if cnt else cnt_why,
                      "launches_per_step": main["launches"],
-                     "issue": issue if issue else {"bound": "alu-issue", "frac": None, "why": cnt_why}},
+                     "issue": issue},
     }
     if st.large:
         flops = sum(2.0 * args.m * s.k_in * s.n_out for s in st.specs)
@@ -452,6 +466,12 @@ def run_ours(args, world, rank, local):
         line["gbs_m%d" % m] = round(st.packed_bytes / (r["ms"] * 1e-3) / 1e9, 3)
     if m1_ms:
         line["pct_of_measured_hbm_m1"] = round(100 * line.get("gbs_m1", gbs) / peak, 2)
+        if args.m != 1:
+            io1 = sum(2 * (s.k_in + s.n_out) + 2 * (s.k_in + 2 * s.n_out) for s in st.specs)
+            line["roofline_m1"] = {"bound": "hbm", "achieved": round((st.packed_bytes + io1) / (m1_ms * 1e-3) / 1e9, 2),
+                                   "peak": peak, "unit": "GB/s", "kernel": "gemv_m1_kernel (one grouped call per layer)",
+                                   "issue": issue_record(1, m1_ms)[0]}
+            line["roofline_m1"]["frac"] = round(line["roofline_m1"]["achieved"] / peak, 4)
         line["step_vs_m1"] = {("m%d" % m): round(r["ms"] / m1_ms, 3) for m, r in results.items() if m != 1}
     for m, ms in chain.items():
         line["us_per_layer_chain_m%d" % m] = round(ms * 1e3 / layers, 3)
