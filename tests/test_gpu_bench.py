@@ -44,7 +44,19 @@ def test_bench_verify_stack_json():
     d = _run_bench("--only", "k")
     _check_common(d, 32)
     assert d["roofline"]["bound"] == "hbm" and d["roofline"]["unit"] == "GB/s"
-    assert d["us_per_layer_m32"] > 0 and d["us_per_layer_m1"] > 0
+    for m in (32, 1, 8, 16):
+        assert d["us_per_layer_m%d" % m] > 0
+    assert "issue" in d["roofline"] and "roofline_m1" in d
+    assert d["e2e"]["eager"]["value"] > 0
+    assert d["config"]["calls"] == "one grouped call per layer"
+
+
+def test_bench_chained_and_separate_json():
+    d = _run_bench("--layers", "2", "--no-extra", "--separate", "--m", "8")
+    _check_common(d, 8)
+    assert d["config"]["calls"] == "one call per matrix"
+    d = _run_bench("--layers", "1")
+    assert d["us_per_layer_chain_m32"] > 0 and d["us_per_layer_chain_m1"] > 0
 
 
 def test_bench_many_row_json():
