@@ -304,6 +304,38 @@ def timed(torch, fn, steps, warmup, barrier):
     return e0.elapsed_time(e1) / steps          # ms per step
 
 
+def time_configs(torch, ex, device, steps, warmup):
+    """Workloads 2-4 (single matrices): each matrix timed as single library
+    calls replayed from one CUDA graph over R copies of its packed words,
+    R chosen so the copies total more than 4x the L2 (no cache reuse between
+    calls); us and packed GB/s per call."""
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    out = {}
+    for cfg, m_list in ((2, (1,)), (3, (1,)), (4, (8, 16))):
+        for m in m_list:
+            for spec in synth.workload(cfg):         # workload 4 at M = 8 takes the first 8 of its 16 rows
+                R = max(2, -(-4 * l2 // spec.packed_bytes))
+                words = torch.stack([synth.splitmix64_words_torch(spec.stream_id, spec.n_words, device)] * R)
+                scale, x, su, sv = synth.small_inputs(spec)
+                dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+                xs, scs, sus, svs = dev(x[:m]), dev(scale), dev(su), dev(sv)
+                y = torch.empty((m, spec.n_out), dtype=torch.float16, device=device)
+                ws = ex.alloc_workspace(m, spec.k_in, spec.n_out, spec.bits, device=device)
+                run = lambda: [ex.gemm(xs, words[r], scs, sus, svs, spec.bits, out=y, workspace=ws) for r in range(R)]
+                run()
+                torch.cuda.synchronize()
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    run()
+                ms = timed(torch, g.replay, max(3, steps // 4), warmup, lambda: None)
+                us = ms * 1e3 / R
+                out[f"c{cfg}.m{m}.{spec.name}"] = {"us": round(us, 2), "gbs": round(spec.packed_bytes / (us * 1e-6) / 1e9, 1),
+                                                   "shape": f"{spec.k_in}x{spec.n_out}", "bits": spec.bits}
+                assert ex.workspace_status(ws) == ex.EXL3_OK
+                del g, words
+    return out
+
+
 def run_ours(args, world, rank, local):
     import torch
     torch.cuda.set_device(local)
@@ -378,6 +410,8 @@ def run_ours(args, world, rank, local):
             chain[m] = rank_max(timed(torch, fn, args.steps, args.warmup, barrier))
             assert ex.workspace_status(st.ws) == ex.EXL3_OK
             del g, st
+
+    configs = time_configs(torch, ex, device, args.steps, args.warmup) if extra and rank == 0 and world == 1 else None
 
     main = results[args.m]
     st = main_stack
@@ -475,6 +509,8 @@ def run_ours(args, world, rank, local):
         line["step_vs_m1"] = {("m%d" % m): round(r["ms"] / m1_ms, 3) for m, r in results.items() if m != 1}
     for m, ms in chain.items():
         line["us_per_layer_chain_m%d" % m] = round(ms * 1e3 / layers, 3)
+    if configs:
+        line["configs_2_to_4"] = configs
     if main["clocks"]:
         line["clocks"] = main["clocks"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -68,9 +68,10 @@ class Stack:
     """The products of ``specs`` (grouped by layer in spec order) at ``m`` rows.
 
     ``weights``: device int32 packed words per spec (e.g. from
-    ``synth.splitmix64_words_torch``).  ``x_rows``: optional callable
-    spec -> (m, k_in) fp16 numpy rows; the default is ``synth.small_inputs``'s
-    rows, repeated when m exceeds them (many-row runs)."""
+    ``synth.splitmix64_words_torch``).  Input rows are ``synth.small_inputs``'s
+    (chained runs: its chain scales), repeated when m exceeds them (many-row
+    runs).  ``large``: use the many-row call (default: m > 32).  ``run_e2e``
+    moves every layer's x and y slices, so it is meant for the sweep."""
 
     def __init__(self, ex, torch, device, m: int, specs, weights, mode: str = "sweep",
                  grouped: bool = True, large: Optional[bool] = None):
