@@ -235,7 +235,11 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     float* zsm = reinterpret_cast<float*>(smem + L::off_z);
 
     const GemmArgs& a = prm.a;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // the warp index broadcast from lane 0: provably warp-uniform, so the values
+    // derived from it (shared-memory descriptors, tensor-memory columns) can stay
+    // in uniform registers, where the tcgen05 instructions take them (measured:
+    // 0.1 fewer instructions per weight, 1-2 % faster)
+    const int warp = __shfl_sync(0xffffffffu, (int)(threadIdx.x >> 5), 0), lane = threadIdx.x & 31;
     const int S = prm.S;
     const int p = blockIdx.x;
     // this CTA's units [b0, b1) in the group's block-major order
