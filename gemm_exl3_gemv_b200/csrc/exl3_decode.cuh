@@ -150,29 +150,28 @@ __device__ __forceinline__ uint32_t window_auto(const uint32_t (&buf)[NW], uint3
 // A lane's share of one tile row of a 128-channel block: 2*BITS consecutive
 // words at `src` (streaming loads: each word is read once).  K = 2, 4: 128-bit
 // loads; K = 3: 64-bit loads (the lane's 24 bytes are 8-byte aligned).
+// The later loads take their offset as an immediate in the instruction (no
+// address arithmetic per load).
 template <int BITS>
 __device__ __forceinline__ void load_lane_words(uint32_t (&w)[2 * BITS], const uint32_t* src)
 {
     if constexpr (BITS == 3) {
-#pragma unroll
-        for (int t = 0; t < 3; ++t) {
-            uint2 v;
-            asm volatile("ld.global.cs.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(src + 2 * t));
-            w[2 * t] = v.x;
-            w[2 * t + 1] = v.y;
-        }
+        asm volatile("ld.global.cs.v2.u32 {%0, %1}, [%6];\n\t"
+                     "ld.global.cs.v2.u32 {%2, %3}, [%6+8];\n\t"
+                     "ld.global.cs.v2.u32 {%4, %5}, [%6+16];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5])
+                     : "l"(src));
+    } else if constexpr (BITS == 4) {
+        asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%8];\n\t"
+                     "ld.global.cs.v4.u32 {%4, %5, %6, %7}, [%8+16];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]), "=r"(w[4]), "=r"(w[5]), "=r"(w[6]),
+                       "=r"(w[7])
+                     : "l"(src));
     } else {
-#pragma unroll
-        for (int t = 0; t < BITS / 2; ++t) {
-            uint4 v;
-            asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "l"(src + 4 * t));
-            w[4 * t] = v.x;
-            w[4 * t + 1] = v.y;
-            w[4 * t + 2] = v.z;
-            w[4 * t + 3] = v.w;
-        }
+        static_assert(BITS == 2, "2, 3 or 4 bits");
+        asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3])
+                     : "l"(src));
     }
 }
 

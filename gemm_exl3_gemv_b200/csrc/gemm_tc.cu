@@ -133,6 +133,20 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
 }
 
+// Warp-wide wait: every lane tries the phase once (one instruction for the
+// warp) and the warp votes; only if the phase is not complete yet does lane 0
+// run the bounded wait and broadcast the outcome.  Nearly nine waits in ten
+// find the phase complete, and this fast path spares them the lane-0 branch,
+// its reconvergence and the broadcast (measured: 0.24 fewer instructions per
+// weight, 3 % faster).  Returns the same value on every lane.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int lane)
+{
+    if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+    int ok = 1;
+    if (lane == 0) ok = wait_or_abort(bar, parity, abort_flag) ? 1 : 0;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
 // zsm[0 .. m*128) = sum of the partial slots (q + g) for q = p_first..p_last,
 // added in that order, by the 256 decoder threads.
 template <int NT>
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         const uint32_t bw = (uint32_t)((warp >> 2) * L::CHUNK + (warp & 3) * 32);
         const uint64_t bdesc0 = sdesc_sw128(smem_u32(smem + L::off_b) + bw, 16, 1024);
         const uint32_t dcol = tmem + (uint32_t)(warp * NT);
-        bool fail0 = false;                                      // lane 0: a wait gave up
+        bool fail0 = false;                                      // a wait gave up (warp-uniform)
         int kk = 0;                                              // CTA unit counter (stages, parities)
         int seg = 0;
         for (long long u0 = b0; u0 < b1; ++seg) {
@@ -344,12 +358,10 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             auto unit = [&](const uint32_t (&wds)[QW], int k, int kq) {
                 const int s = kq & (kAStages - 1), bs = kq & (kBStages - 1);
                 const uint32_t ph = (uint32_t)(kq / kAStages) & 1u, bph = (uint32_t)(kq / kBStages) & 1u;
-                // lane 0 waits for the MMA that last read this stage; the shuffle
-                // then orders every lane's stores after it
-                int okw = 1;
-                if (lane == 0)
-                    okw = !fail0 && (kq < kAStages || wait_or_abort(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag));
-                if (!__shfl_sync(0xffffffffu, okw, 0)) ok = false;
+                // every lane sees the MMA that last read this stage complete before
+                // it stores into the stage
+                if (fail0 || !(kq < kAStages || warp_wait(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag, lane)))
+                    ok = false;
                 if (!ok) return;
                 uint32_t buf[QW + 1];
                 buf[0] = __shfl_sync(0xffffffffu, wds[QW - 1], src_prev);
@@ -362,16 +374,14 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 });
                 fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
                 __syncwarp();
-                int okb = 1;
-                if (lane == 0) okb = wait_or_abort(&bfull[bs], bph, abort_flag) ? 1 : 0;
-                if (__shfl_sync(0xffffffffu, okb, 0)) {
+                if (warp_wait(&bfull[bs], bph, abort_flag, lane)) {
                     tc_fence_after();
                     const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
                     mma_f16_ss_elect(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
                     mma_commit_elect(&aempty[warp * kAStages + s]);
                     mma_commit_elect(&bempty[bs]);
-                } else if (lane == 0) {
-                    fail0 = true;                        // seen by the whole warp at its next unit
+                } else {
+                    fail0 = true;                        // warp-uniform: ends the warp's units
                 }
             };
             uint32_t wa[QW], wb[QW];
