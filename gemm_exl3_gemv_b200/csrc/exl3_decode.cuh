@@ -138,12 +138,13 @@ __device__ __forceinline__ uint32_t window_bytes(const uint32_t (&buf)[NW], uint
 
 // Window isolation chosen per bit width (measured on B200): byte-aligned
 // reads from shifted words for 2 and 4 bits; for 3 bits (windows at every
-// bit offset) every second non-aligned window on the FMA pipe.  R is the
-// weight's index in the run, P its window's start bit in `buf`.
+// bit offset) every third non-aligned window on the FMA pipe (every second:
+// up to 2 % slower).  R is the weight's index in the run, P its window's
+// start bit in `buf`.
 template <int BITS, int R, int P, int NW>
 __device__ __forceinline__ uint32_t window_auto(const uint32_t (&buf)[NW], uint32_t two16)
 {
-    if constexpr (BITS == 3) return window_of<P, NW, (R % 2) == 0>(buf, two16);
+    if constexpr (BITS == 3) return window_of<P, NW, (R % 3) == 0>(buf, two16);
     else return window_bytes<P, NW>(buf, two16);
 }
 

@@ -88,6 +88,23 @@ __device__ __forceinline__ void mma_commit_elect(uint64_t* bar)
         : "memory");
 }
 
+// The MMA and two commits (each arrives once every MMA the thread issued so
+// far has completed) issued by one elected lane under a single election.
+__device__ __forceinline__ void mma_f16_ss_commit2_elect(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                                         uint32_t idesc, uint32_t accumulate, uint64_t* bar0,
+                                                         uint64_t* bar1)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%5];\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%6];\n\t}" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(smem_u32(bar0)), "r"(smem_u32(bar1))
+        : "memory");
+}
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar)
 {

@@ -377,9 +377,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                 if (warp_wait(&bfull[bs], bph, abort_flag, lane)) {
                     tc_fence_after();
                     const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
-                    mma_f16_ss_elect(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u);
-                    mma_commit_elect(&aempty[warp * kAStages + s]);
-                    mma_commit_elect(&bempty[bs]);
+                    mma_f16_ss_commit2_elect(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u,
+                                             &aempty[warp * kAStages + s], &bempty[bs]);
                 } else {
                     fail0 = true;                        // warp-uniform: ends the warp's units
                 }
