@@ -153,6 +153,24 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
     };
     grid_dep_launch();                     // the next product may start loading its weights
     bool first_seg = true;
+    // the first words of this warp's next segment, loaded before the current
+    // segment's reduction and epilogue so that their latency hides behind them
+    // (measured: 2.4 % off the single-row layer call)
+    uint32_t wa[QW];
+    auto seg_load = [&](long long us) {
+        const MemView mv = member_of_unit(a, us);
+        const int T = mv.k_in / 16;
+        const int gl = (int)((us - mv.u0) / T);
+        const long long ublk = mv.u0 + (long long)gl * T;
+        const int rs = (int)(us - ublk);
+        const int re = (int)((ublk + T < b1 ? ublk + T : b1) - ublk);
+        if (re - rs > warp) {
+            const int tiles_n = mv.n_out / 16;
+            const uint32_t* s0 = mv.packed + ((size_t)(rs + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
+            load_lane_words_checked<BITS>(wa, s0, mv.packed, (size_t)T * tiles_n * TW, status);
+        }
+    };
+    if (b0 < b1) seg_load(b0);
 
     for (long long u = b0; u < b1;) {
         // ---- segment: block g (group numbering), tile rows [r0, r1) of its member ----
@@ -180,8 +198,7 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
         const int kb_lo = r0 >> 3, kb_hi = (r1 + 7) >> 3;             // 128-row input blocks touched
         const int nrow = r1 - r0;
         const int nw = nrow > warp ? (nrow - warp + kM1Warps - 1) / kM1Warps : 0;
-        uint32_t wa[QW], wb[QW];
-        if (nw > 0) load_lane_words_checked<BITS>(wa, src, wbase, n_words, status);   // in flight during the rotation
+        uint32_t wb[QW];
         if (first_seg) grid_dep_wait();    // weights are never written; x, y, workspace only after this
         first_seg = false;
 
@@ -230,6 +247,7 @@ __global__ void __launch_bounds__(kM1Threads, kM1MinBlocks<BITS>)
             for (int c = 0; c < 16; ++c) accf[c] = add_pair_f32(accf[c], acc[c]);
         }
 
+        if (u < b1) seg_load(u);                                       // in flight during the reduction
         // ---- reduce: the 4 quarters of a tile, then the 8 warps (fixed order) ----
 #pragma unroll
         for (int c = 0; c < 16; ++c) {

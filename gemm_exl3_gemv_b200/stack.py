@@ -18,7 +18,9 @@ Two ways to chain the layer's seven matrices (q, k, v, o, gate, up, down):
   layer input h (one sibling call, ``exl3_gemm_siblings``), o takes q's output
   (the stand-in for attention is the identity), down takes up's output (the
   stand-in for the activation is the identity), and down's output is the next
-  layer's h.  Three dependent steps per layer.
+  layer's h.  o and down depend only on the sibling call, so with
+  ``grouped=True`` they run as one grouped call: two dependent steps per
+  layer (three with ``grouped=False``).
 
 Buffers: inputs and outputs of all products live in one flat device buffer
 each (x and y), a layer's slices contiguous, so an end-to-end step moves one
@@ -80,7 +82,7 @@ class Stack:
         self.ex, self.torch, self.device = ex, torch, device
         self.m, self.mode = m, mode
         self.large = (m > 32) if large is None else large
-        self.grouped = grouped and not self.large and mode == "sweep"
+        self.grouped = grouped and not self.large
         self.specs = list(specs)
         x_off, y_off, xo, yo = [], [], 0, 0
         for s in self.specs:
@@ -138,8 +140,11 @@ class Stack:
             if self.mode == "chain":
                 P = {p.kind: p for p in lay.products}
                 calls.append(("siblings", [P["q"], P["k"], P["v"], P["gate"], P["up"]]))
-                calls.append(("single", P["o"]))
-                calls.append(("single", P["down"]))
+                if self.grouped:
+                    calls.append(("grouped", [P["o"], P["down"]]))
+                else:
+                    calls.append(("single", P["o"]))
+                    calls.append(("single", P["down"]))
             elif self.grouped:
                 calls.append(("grouped", lay.products))
             else:
@@ -196,8 +201,13 @@ class Stack:
             ex.gemm_siblings(h, q.su, [(p.packed, p.scale, p.sv) for p in sib], q.spec.bits,
                              outs=[p.y for p in sib], workspace=self.ws)
             o, d = P["o"], P["down"]
-            ex.gemm(P["q"].y, o.packed, o.scale, o.su, o.sv, o.spec.bits, out=o.y, workspace=self.ws)
-            ex.gemm(P["up"].y, d.packed, d.scale, d.su, d.sv, d.spec.bits, out=d.y, workspace=self.ws)
+            if self.grouped:
+                ex.gemm_grouped([(P["q"].y, o.packed, o.scale, o.su, o.sv, o.y),
+                                 (P["up"].y, d.packed, d.scale, d.su, d.sv, d.y)],
+                                o.spec.bits, workspace=self.ws)
+            else:
+                ex.gemm(P["q"].y, o.packed, o.scale, o.su, o.sv, o.spec.bits, out=o.y, workspace=self.ws)
+                ex.gemm(P["up"].y, d.packed, d.scale, d.su, d.sv, d.spec.bits, out=d.y, workspace=self.ws)
             return
         if self.grouped:
             ex.gemm_grouped([(p.x, p.packed, p.scale, p.su, p.sv, p.y) for p in lay.products],

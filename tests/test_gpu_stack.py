@@ -85,7 +85,8 @@ def _chain_depth(spec):
 
 
 @pytest.mark.parametrize("m", [1, 32])
-def test_graphed_chain_matches_composed_oracle(oracle_mod, m):
+@pytest.mark.parametrize("grouped", [True, False])
+def test_graphed_chain_matches_composed_oracle(oracle_mod, m, grouped):
     """Tolerance: each product meets the per-product bound (rel-L2 1e-3,
     max-abs 1e-2) on its own inputs (the other tests).  In a chain the input
     of product d is the library's fp16 output of product d - 1, which already
@@ -95,7 +96,8 @@ def test_graphed_chain_matches_composed_oracle(oracle_mod, m):
     rel-L2 <= d * 1e-3 and max-abs <= d * 1e-2 at depth d."""
     import gpu_helpers
     layers = 2
-    st = _stack(m, layers, "chain", False)
+    st = _stack(m, layers, "chain", grouped)
+    assert len(st._calls()) == layers * (2 if grouped else 3)
     _replay(st)
     ref = _oracle_chain(oracle_mod, st.specs, m, layers)
     for p in st.products:
@@ -105,7 +107,7 @@ def test_graphed_chain_matches_composed_oracle(oracle_mod, m):
         rel = np.linalg.norm(got - r) / np.linalg.norm(r)
         mx = np.abs(got - r).max()
         assert np.all(np.isfinite(got)), p.spec.name
-        assert rel <= d * gpu_helpers.REL_L2, f"chain {p.spec.name} m={m} depth {d}: rel-L2 {rel:.3e}"
-        assert mx <= d * gpu_helpers.MAX_ABS, f"chain {p.spec.name} m={m} depth {d}: max-abs {mx:.3e}"
+        assert rel <= d * gpu_helpers.REL_L2, f"chain {p.spec.name} m={m} grouped={grouped} depth {d}: rel-L2 {rel:.3e}"
+        assert mx <= d * gpu_helpers.MAX_ABS, f"chain {p.spec.name} m={m} grouped={grouped} depth {d}: max-abs {mx:.3e}"
     # the chain is carried: layer 1's input is layer 0's down output
     assert np.abs(ref["l1.down"]).max() > 0
