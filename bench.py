@@ -465,7 +465,7 @@ def run_ours(args, world, rank, local):
         "e2e": {"value": round(world * st.packed_bytes / (main["e2e_ms"] * 1e-3) / 1e9, 3), "unit": UNIT,
                 "h2d_bytes_per_step": st.h2d, "d2h_bytes_per_step": st.d2h,
                 "ms_per_step": round(main["e2e_ms"], 4),
-                "pipeline": "per layer: H2D stream -> products -> D2H stream, overlapped; " + main["e2e_launch"],
+                "pipeline": "inputs up in growing chunks of layers, products, outputs down in shrinking chunks, on three streams, overlapped; " + main["e2e_launch"],
                 "eager": {"value": round(world * st.packed_bytes / (main["e2e_eager_ms"] * 1e-3) / 1e9, 3),
                           "ms_per_step": round(main["e2e_eager_ms"], 4),
                           "launch": "eager: every library call through the binding and the C ABI each step"}},

@@ -221,30 +221,58 @@ class Stack:
         for li in range(len(self.layers)):
             self.run_layer(li)
 
+    def _copy_chunks(self, growth: float = 1.6):
+        """Layer ranges [a, b) whose inputs go up in one copy: 1, 1, 2, 3, 5, ...
+        layers, each range growing by ``growth`` -- slow enough that a range has
+        landed by the time the products reach it (a layer's inputs copy in about
+        half the time its products take)."""
+        n = len(self.layers)
+        b = [0, 1]
+        while b[-1] < n:
+            b.append(min(n, int(b[-1] * growth) + 1))
+        return list(zip(b[:-1], b[1:]))
+
     def run_e2e(self):
-        """One end-to-end step from pinned host buffers: per layer, its inputs go
-        up on one stream, its products run on the current stream, its outputs
-        come down on a third, so the copies of one layer overlap the products of
-        its neighbours.  Every copy is inside the step."""
+        """One end-to-end step from pinned host buffers: the inputs go up on one
+        stream in growing chunks of layers (``_copy_chunks``), the products run
+        on the current stream, the outputs come down on a third stream in
+        chunks that shrink towards the last layer, so the copies overlap the
+        products and the step ends one layer's output copy after its last
+        product.  Every copy is inside the step.  Chunks rather than one copy
+        per layer: each cross-stream wait in front of a product costs the
+        overlap of that product with the previous one's tail (measured with 64
+        layers at M = 32: 7.94 ms per step with a wait per layer, 7.66 ms with
+        nine)."""
         torch = self.torch
+        n = len(self.layers)
+        for prev, lay in zip(self.layers, self.layers[1:]):
+            assert lay.x0 == prev.x1 and lay.y0 == prev.y1, "layer slices must be contiguous"
         cs = torch.cuda.current_stream()
         start = torch.cuda.Event()
         start.record(cs)
         self.s_in.wait_event(start)
         self.s_out.wait_event(start)
-        for li, lay in enumerate(self.layers):
-            xs, ys = slice(lay.x0, lay.x1), slice(lay.y0, lay.y1)
-            with torch.cuda.stream(self.s_in):
+        landed = {}
+        with torch.cuda.stream(self.s_in):
+            for a, b in self._copy_chunks():
+                xs = slice(self.layers[a].x0, self.layers[b - 1].x1)
                 self.x_dev[xs].copy_(self.x_pin[xs], non_blocking=True)
-                ev_in = torch.cuda.Event()
-                ev_in.record(self.s_in)
-            cs.wait_event(ev_in)
+                ev = torch.cuda.Event()
+                ev.record(self.s_in)
+                landed[a] = ev
+        out_chunks = {n - 1 - a: (n - b, n - a) for a, b in self._copy_chunks()}   # mirrored
+        for li in range(n):
+            if li in landed:
+                cs.wait_event(landed[li])
             self.run_layer(li)
-            ev_out = torch.cuda.Event()
-            ev_out.record(cs)
-            self.s_out.wait_event(ev_out)
-            with torch.cuda.stream(self.s_out):
-                self.y_pin[ys].copy_(self.y_dev[ys], non_blocking=True)
+            if li in out_chunks:
+                a, b = out_chunks[li]
+                ev = torch.cuda.Event()
+                ev.record(cs)
+                self.s_out.wait_event(ev)
+                with torch.cuda.stream(self.s_out):
+                    ys = slice(self.layers[a].y0, self.layers[b - 1].y1)
+                    self.y_pin[ys].copy_(self.y_dev[ys], non_blocking=True)
         cs.wait_stream(self.s_in)
         cs.wait_stream(self.s_out)
 

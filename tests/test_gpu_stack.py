@@ -55,6 +55,33 @@ def test_graphed_stack_slice_matches_oracle(oracle_mod, m, grouped):
         check_close(p.y.cpu().numpy(), ref, f"{p.spec.name} m={m} grouped={grouped}")
 
 
+@pytest.mark.parametrize("m", [32, 1])
+def test_graphed_end_to_end_matches_oracle(oracle_mod, m):
+    """The bench's end-to-end step (inputs copied up from pinned host memory
+    in chunks of layers, outputs copied down in chunks, as one CUDA graph):
+    the device inputs and outputs are poisoned first, so every host output
+    must come from this step's copies and products.  Five layers, so that
+    both copy directions include a multi-layer chunk."""
+    import torch
+    st = _stack(m, 5, "sweep", True)
+    assert any(b - a > 1 for a, b in st._copy_chunks())
+    g = st.capture(st.run_e2e)
+    st.x_dev.fill_(float("nan"))
+    st.y_dev.fill_(float("nan"))
+    st.y_pin.fill_(float("nan"))
+    g.replay()
+    torch.cuda.synchronize()
+    from gemm_exl3_gemv_b200 import exl3 as ex
+    assert ex.workspace_status(st.ws) == ex.EXL3_OK
+    del g
+    for p in st.products:
+        inp = synth.make_inputs(p.spec)
+        ref = oracle_mod.gemm(inp.x[:m], inp.packed, inp.scale, inp.su, inp.sv, p.spec.k_in, p.spec.n_out, p.spec.bits)
+        off = (p.y.data_ptr() - st.y_dev.data_ptr()) // 2
+        host = st.y_pin[off:off + m * p.spec.n_out].view(m, p.spec.n_out).numpy()
+        check_close(host, ref, f"end-to-end {p.spec.name} m={m}")
+
+
 def _oracle_chain(oracle_mod, specs, m, layers):
     """The chained step composed from oracle products, with the activations
     rounded to fp16 between products (as the library stores them)."""

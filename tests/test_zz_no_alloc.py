@@ -1,8 +1,9 @@
 """exl3_gemv_noalloc: the single-row product for callers that cannot allocate
 device memory (no workspace argument; the library's own fixed scratch array
-is used instead).  Checked through the C ABI against exl3_gemv with a
-caller-allocated workspace, on two calls in a row (the scratch array keeps
-the previous call's contents, so the second call checks that the entry point
+is used instead).  Checked through the C ABI against the fp64 oracle and
+against exl3_gemv with a caller-allocated workspace (bitwise: the same
+kernel and split), on two calls in a row (the scratch array keeps the
+previous call's contents, so the second call checks that the entry point
 clears what must start at zero).  Kept in a file of its own that pytest
 collects last."""
 import ctypes
@@ -27,19 +28,22 @@ def _noalloc(ex, x, packed, scale, su, sv, y, k, n, bits):
 
 
 @pytest.mark.parametrize("idx", [0, 1])
-def test_noalloc_matches_workspace_gemv_twice(idx):
+def test_noalloc_matches_oracle_and_workspace_gemv_twice(oracle_mod, idx):
     import torch
     from gemm_exl3_gemv_b200 import exl3 as ex
     spec = [synth.workload(2)[0], synth.workload(3)[2]][idx]          # o_proj 5120x5120; down 17408x5120
     inp = synth.make_inputs(spec)
     x, packed, scale, su, sv = (to_dev(a) for a in (inp.x[0], inp.packed, inp.scale, inp.su, inp.sv))
-    ref = ex.gemm(x, packed, scale, su, sv, spec.bits, fp32=True).cpu().numpy()
+    ws_y = ex.gemm(x, packed, scale, su, sv, spec.bits, fp32=True).cpu().numpy()
+    ref = oracle_mod.gemm(inp.x[:1], inp.packed, inp.scale, inp.su, inp.sv, spec.k_in, spec.n_out, spec.bits)[0]
     for call in range(2):
         y = torch.full((spec.n_out,), float("nan"), dtype=torch.float32, device="cuda")
         st = _noalloc(ex, x, packed, scale, su, sv, y, spec.k_in, spec.n_out, spec.bits)
         assert st == ex.EXL3_OK, ex.lib.exl3_status_string(st)
         torch.cuda.synchronize()
-        check_close(y.cpu().numpy(), ref, f"noalloc call {call}")
+        got = y.cpu().numpy()
+        check_close(got, ref, f"noalloc call {call} vs oracle")
+        assert np.array_equal(got, ws_y), f"noalloc call {call}: differs from exl3_gemv with a workspace"
 
 
 def test_noalloc_rejects_problem_beyond_scratch():
