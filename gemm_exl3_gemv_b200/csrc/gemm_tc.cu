@@ -10,25 +10,29 @@
 //   * A pre-pass writes xt = H(su .* x) once per call into the workspace, fp16,
 //     laid out as the MMA's B operand (K-major, 128-byte swizzle), m padded to
 //     NT = 16 or 32 rows with zeros.
-//   * Unit = one 128-row block of K_in for one 128-channel output block: 8
-//     tile rows, 16384 weights.  Two ways to cut the units over the CTAs (two
-//     per SM), chosen per shape by a small cost model (see TcParams):
-//     clusters of S CTAs per output block that add their partial sums through
-//     distributed shared memory, or a stream-K cut with workspace partials.
-//   * Eight decoder warps.  Warp w decodes tile row w of every unit: lane l
-//     takes quarter l%4 of tile l/4 (64 consecutive weights) from its words,
-//     loaded straight from HBM into registers one unit ahead (coalesced: the
-//     warp reads the tile row's 256*K contiguous bytes).  The two fp16 halves
-//     of each 3INST word are added once (RNE: the exact decoded weight) and
-//     stored into the warp's own A stage (128 channels x 16 k, MN-major,
-//     128-byte swizzle).  The warp then issues the MMA itself (one elected
-//     lane, from converged code) -- tcgen05.mma kind::f16, M = 128 channels,
-//     N = NT rows, K = 16 -- into the warp's own tensor-memory accumulator
-//     (so the accumulation order is fixed), and commits it to the stage's
-//     barrier.  A warp waits only for
-//     its own stage (two units back) and for the unit's xt.
+//   * Unit = one block of 128 RPW rows of K_in for one 128-channel output
+//     block: 8 RPW tile rows.  RPW = 2 (256-row units) when every K_in of the
+//     call is a multiple of 256, else 1.  Two ways to cut the units over the
+//     CTAs (two per SM), chosen per shape by a small cost model (see
+//     TcParams): clusters of S CTAs per output block that add their partial
+//     sums through distributed shared memory, or a stream-K cut with
+//     workspace partials.
+//   * Eight decoder warps.  Warp w decodes tile rows w (and w + 8) of every
+//     unit: lane l takes quarter l%4 of tile l/4 (64 consecutive weights) from
+//     its words, loaded straight from HBM into registers one tile row ahead
+//     (coalesced: the warp reads the tile row's 256*K contiguous bytes).  The
+//     two fp16 halves of each 3INST word are added once (RNE: the exact
+//     decoded weight) and stored into the warp's own A stage (128 channels x
+//     16 k per tile row, MN-major, 128-byte swizzle).  The warp then issues
+//     the unit's MMAs itself (one elected lane, from converged code) --
+//     tcgen05.mma kind::f16, M = 128 channels, N = NT rows, K = 16 -- into its
+//     own tensor-memory accumulator (so the accumulation order is fixed), and
+//     commits them to the stage's barrier.  A warp waits only for its own
+//     stage and for the unit's xt; with two tile rows per unit it hands off
+//     half as often (measured: 3 % off a grouped layer call).
 //   * A ninth warp streams each unit's xt (1-D bulk copies + mbarrier) into a
-//     four-stage ring shared by the eight decoders.
+//     ring shared by the eight decoders (four stages of 128 rows, or two of
+//     256).
 //   * End of a block's share: the CTA reads all eight accumulators
 //     (tcgen05.ld) and adds them in a fixed order; the partial sums of a block
 //     split over several CTAs meet in rank / CTA order -- fixed, so results
@@ -61,32 +65,39 @@ namespace {
 constexpr int kDec = 8;                        // decoder warps (one accumulator each)
 constexpr int kProdWarp = kDec;                // warp 8: xt chunk producer
 constexpr int kTcThreads = 32 * (kDec + 1);
-constexpr int kAStages = 2;                    // A stages per decoder warp
-constexpr int kBStages = 4;                    // xt unit stages (shared by the eight decoders)
-constexpr int kABytes = 4096;                  // one tile row of A: 128 channels x 16 k, fp16
+constexpr int kATile = 4096;                   // one tile row of A: 128 channels x 16 k, fp16
 constexpr int kCtasPerSm = 2;
 constexpr int kSms = 148;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
-template <int NT>
+// RPW tile rows per decoder warp per unit: a unit is 128 * RPW input rows.
+// RPW = 1: two A stages of one tile row per warp, four xt stages; RPW = 2:
+// one A stage of two tile rows per warp (the first half tile row is decoded
+// into registers while the previous unit's MMAs finish), two xt stages.
+template <int NT, int RPW>
 struct TcLayout {
+    static constexpr int AST = RPW == 1 ? 2 : 1;              // A stages per decoder warp
+    static constexpr int BST = RPW == 1 ? 4 : 2;              // xt unit stages (shared by the decoders)
+    static constexpr int ABYTES = RPW * kATile;               // one A stage
     static constexpr int CHUNK = NT * 128;                    // xt bytes per 64 input rows
-    static constexpr int BUNIT = 2 * CHUNK;                   // xt bytes per unit (128 rows)
+    static constexpr int BUNIT = 2 * RPW * CHUNK;             // xt bytes per unit
     static constexpr int TMEM_COLS = kDec * NT;               // one NT-column accumulator per decoder
-    static constexpr int off_a = 0;                           // [kDec][kAStages] A stages
+    static constexpr int off_a = 0;                           // [kDec][AST] A stages
     static constexpr int off_z = off_a;                       // z [NT][128] fp32, over the A stages (segment end)
-    static constexpr int off_b = off_a + kDec * kAStages * kABytes;
-    static constexpr int off_bar = off_b + kBStages * BUNIT;
-    // aempty[kDec][kAStages], bfull[kBStages], bempty[kBStages], segdone, lastbar
-    static constexpr int nbar = kDec * kAStages + 2 * kBStages + 2;
+    static constexpr int off_b = off_a + kDec * AST * ABYTES;
+    static constexpr int off_bar = off_b + BST * BUNIT;
+    // aempty[kDec][AST], bfull[BST], bempty[BST], segdone, lastbar
+    static constexpr int nbar = kDec * AST + 2 * BST + 2;
     static constexpr int off_misc = off_bar + nbar * 8;
     static constexpr int total = off_misc + 64 + 1024;       // + slack to align the base to 1024
     static_assert(off_b % 1024 == 0 && off_z % 16 == 0 && off_bar % 8 == 0, "layout");
-    static_assert(NT * 128 * 4 <= kDec * kAStages * kABytes, "z fits over the A stages");
+    static_assert(NT * 128 * 4 <= kDec * AST * ABYTES, "z fits over the A stages");
+    static_assert((BST & (BST - 1)) == 0, "power of two");
     static_assert(TMEM_COLS == 128 || TMEM_COLS == 256, "tensor memory (power of two, two CTAs per SM)");
     // at most two CTAs fit on an SM, so their accumulators always fit in its 512 columns
     static_assert(3 * total > 227 * 1024, "a third CTA per SM must not fit");
-    static_assert(kCtasPerSm * total <= 227 * 1024, "two CTAs per SM");
+    // 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
+    static_assert(kCtasPerSm * (total + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 // Two ways to cut the G x C units (output block g, 128-row input block c):
@@ -231,18 +242,64 @@ __device__ __forceinline__ void finish_row(const GemmArgs& a, int g, int mm, con
     finish_row_regs(a, g, mm, z, lane);
 }
 
-template <int BITS, int NT>
+// decode_quarter_to_a restricted to its 16-byte chunks RE0 .. RE1 - 1 (chunk
+// RE = 2 r + e: row r of the quarter, channels 8e .. 8e + 7); the same
+// arithmetic and window forms per weight.
+template <int BITS, int RE0, int RE1, int NW, typename Put>
+__device__ __forceinline__ void decode_quarter_chunks(const uint32_t (&buf)[NW], const uint32_t (&soff)[2][2],
+                                                      uint32_t two16, Put&& put)
+{
+    auto body = [&](auto R, auto E) {
+        constexpr int r = decltype(R)::value, e = decltype(E)::value;
+        auto pair = [&](auto Cc) -> uint32_t {
+            constexpr int c = decltype(Cc)::value;
+            constexpr int ia = 16 * r + 8 * e + 2 * c, ib = ia + 1;
+            const uint32_t ma = inst3(window_auto<BITS, ia, (ia + 1) * BITS + 16>(buf, two16));
+            const uint32_t mb = inst3(window_auto<BITS, ib, (ib + 1) * BITS + 16>(buf, two16));
+            return weight_pair_h(ma, mb);
+        };
+        put(soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
+            pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
+            pair(std::integral_constant<int, 3>{}));
+    };
+    [&]<int... RE>(std::integer_sequence<int, RE...>) {
+        (body(std::integral_constant<int, (RE0 + RE) / 2>{}, std::integral_constant<int, (RE0 + RE) % 2>{}), ...);
+    }(std::make_integer_sequence<int, RE1 - RE0>{});
+}
+
+// Two MMAs into one accumulator (the second always accumulating) and two
+// commits, issued by one elected lane under a single election.
+__device__ __forceinline__ void mma2_f16_ss_commit2_elect(uint32_t d_tmem, uint64_t adesc0, uint64_t bdesc0,
+                                                          uint64_t adesc1, uint64_t bdesc1, uint32_t idesc,
+                                                          uint32_t accumulate, uint64_t* bar0, uint64_t* bar1)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "elect.sync _|e, 0xffffffff;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %5, p;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %5, 1;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%7];\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%8];\n\t}" ::"r"(d_tmem),
+        "l"(adesc0), "l"(bdesc0), "l"(adesc1), "l"(bdesc1), "r"(idesc), "r"(accumulate), "r"(smem_u32(bar0)),
+        "r"(smem_u32(bar1))
+        : "memory");
+}
+
+template <int BITS, int NT, int RPW>
 __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParams prm)
 {
-    using L = TcLayout<NT>;
+    using L = TcLayout<NT, RPW>;
+    constexpr int AST = L::AST, BST = L::BST;
+    constexpr int KU = 128 * RPW;                             // input rows per unit
     constexpr int TW = 8 * BITS, QW = 2 * BITS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::off_bar);
-    uint64_t* aempty = bar;                                   // [kDec][kAStages]: the stage's MMA completed
-    uint64_t* bfull = aempty + kDec * kAStages;               // [kBStages]: xt unit landed
-    uint64_t* bempty = bfull + kBStages;                      // [kBStages]: all 8 MMAs on it completed
-    uint64_t* segdone = bempty + kBStages;                    // every accumulator final
+    uint64_t* aempty = bar;                                   // [kDec][AST]: the stage's MMAs completed
+    uint64_t* bfull = aempty + kDec * AST;                    // [BST]: xt unit landed
+    uint64_t* bempty = bfull + BST;                           // [BST]: all 8 warps' MMAs on it completed
+    uint64_t* segdone = bempty + BST;                         // every accumulator final
     uint64_t* lastbar = segdone + 1;                          // every MMA of the CTA completed
     int* misc = reinterpret_cast<int*>(smem + L::off_misc);   // [0] tmem base, [1] abort
     volatile int* abort_flag = misc + 1;
@@ -261,7 +318,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     if (S > 0) {
         const int gc = p / S, rc = p % S;
         const MemView cm = member_of_block(a, gc);
-        const int C = cm.k_in / 128;
+        const int C = cm.k_in / KU;
         const long long ublk = cm.u0 + (long long)cm.gl * C;
         b0 = ublk + (long long)rc * C / S;
         b1 = ublk + (long long)(rc + 1) * C / S;
@@ -271,8 +328,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     }
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kDec * kAStages; ++i) mbar_init(&aempty[i], 1);
-        for (int i = 0; i < kBStages; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kDec); }
+        for (int i = 0; i < kDec * AST; ++i) mbar_init(&aempty[i], 1);
+        for (int i = 0; i < BST; ++i) { mbar_init(&bfull[i], 1); mbar_init(&bempty[i], kDec); }
         mbar_init(segdone, kDec);
         mbar_init(lastbar, kDec);
         misc[1] = 0;
@@ -292,7 +349,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
     if (warp == kProdWarp) {
         grid_dep_wait();               // xt is written by the pre-pass
         // ------------------------------------------------- xt producer ---
-        // xt of unit (g, c) is chunks 2c, 2c+1: BUNIT contiguous bytes.
+        // xt of unit (g, c) is chunks 2 RPW c .. 2 RPW c + 2 RPW - 1: BUNIT contiguous bytes.
         // A nonzero injection word v (tests of the timeout path) lets only the
         // CTA's first v - 1 xt copies through, so the decoders' wait for the
         // next one runs out (with MMAs of the earlier units possibly in flight).
@@ -301,10 +358,10 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         if (lane == 0) {
             int kk = 0;
             for (long long u = b0; u < b1 && kk < allowed; ++u, ++kk) {
-                const int s = kk & (kBStages - 1);
-                if (kk >= kBStages && !wait_or_abort(&bempty[s], (uint32_t)(kk / kBStages - 1) & 1u, abort_flag)) break;
+                const int s = kk & (BST - 1);
+                if (kk >= BST && !wait_or_abort(&bempty[s], (uint32_t)(kk / BST - 1) & 1u, abort_flag)) break;
                 const MemView um = member_of_unit(a, u);
-                const int c = (int)((u - um.u0) % (um.k_in / 128));
+                const int c = (int)((u - um.u0) % (um.k_in / KU));
                 if (!guard(um.xt0 + (size_t)(c + 1) * L::BUNIT <= prm.xt_bytes, prm.status)) break;
                 mbar_arrive_expect_tx(&bfull[s], L::BUNIT);
                 bulk_g2s(smem + L::off_b + s * L::BUNIT, prm.xt + um.xt0 + (size_t)c * L::BUNIT, L::BUNIT, &bfull[s]);
@@ -312,8 +369,8 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             // every issued copy lands before the CTA can exit (a no-op wait in
             // a normal run: the decoders have consumed them)
             const int issued = kk;
-            for (int v = issued > kBStages ? issued - kBStages : 0; v < issued; ++v)
-                (void)mbar_wait_bounded(&bfull[v & (kBStages - 1)], (uint32_t)(v / kBStages) & 1u, 100000000ull);
+            for (int v = issued > BST ? issued - BST : 0; v < issued; ++v)
+                (void)mbar_wait_bounded(&bfull[v & (BST - 1)], (uint32_t)(v / BST) & 1u, 100000000ull);
         }
     } else {
         // --------------------------------------------- decoder warps ---
@@ -325,13 +382,13 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         uint32_t soff[2][2];
         lane_soff(lane, soff);
         constexpr uint32_t idesc = idesc_f16_amn(128, NT);
-        static_assert(kAStages == 2, "A stage index = unit counter & 1");
-        static_assert((kBStages & (kBStages - 1)) == 0, "power of two");
-        const uint32_t ast0 = smem_u32(smem + L::off_a + (warp * kAStages + 0) * kABytes);
-        const uint32_t ast1 = smem_u32(smem + L::off_a + (warp * kAStages + 1) * kABytes);
+        const uint32_t ast0 = smem_u32(smem + L::off_a + (warp * AST + 0) * L::ABYTES);
+        // RPW = 1: the second A stage; RPW = 2: the stage's second tile row
+        const uint32_t ast1 = RPW == 1 ? smem_u32(smem + L::off_a + (warp * AST + 1) * L::ABYTES) : ast0 + kATile;
         const uint64_t adesc0 = sdesc_sw128(ast0, 1024, 2048), adesc1 = sdesc_sw128(ast1, 1024, 2048);
-        // this warp's tile row is rows 16*warp .. +15 of a unit: chunk warp/4, 32 bytes per 16 rows;
-        // stage bs adds bs * BUNIT to the start address (no carry out of its 14-bit field: smem < 256 KB)
+        // this warp's tile rows are rows 16 (warp + 8 j) .. +15 of a unit (j < RPW): chunk warp/4 + 2 j,
+        // 32 bytes per 16 rows; stage bs adds bs * BUNIT to the start address (no carry out of its
+        // 14-bit field: smem < 256 KB)
         const uint32_t bw = (uint32_t)((warp >> 2) * L::CHUNK + (warp & 3) * 32);
         const uint64_t bdesc0 = sdesc_sw128(smem_u32(smem + L::off_b) + bw, 16, 1024);
         const uint32_t dcol = tmem + (uint32_t)(warp * NT);
@@ -340,7 +397,7 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
         int seg = 0;
         for (long long u0 = b0; u0 < b1; ++seg) {
             const MemView sib = member_of_unit(a, u0);                 // the matrix holding unit u0
-            const int C = sib.k_in / 128;                              // units per block of this matrix
+            const int C = sib.k_in / KU;                               // units per block of this matrix
             const int gl = (int)((u0 - sib.u0) / C);
             const int g = sib.g0 + gl;                                 // group block index
             const long long ublk = sib.u0 + (long long)gl * C;         // the block's first unit
@@ -348,19 +405,22 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
             const long long u1 = (ublk + C < b1) ? ublk + C : b1;
             const int nseg = (int)(u1 - u0);
             const int tiles_n = sib.n_out / 16;
+            const size_t rstep = (size_t)8 * tiles_n * TW;        // words between tile rows w and w + 8
             const uint32_t* src =
-                sib.packed + ((size_t)(8 * c0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
-            const size_t unit_step = (size_t)8 * tiles_n * TW;    // words between consecutive units
-            const size_t n_words = (size_t)C * 8 * tiles_n * TW;
+                sib.packed + ((size_t)(8 * RPW * c0 + warp) * tiles_n + 8 * (size_t)gl) * TW + (size_t)lane * QW;
+            const size_t unit_step = (size_t)RPW * rstep;        // words between consecutive units
+            const size_t n_words = (size_t)C * unit_step;
             bool ok = true;                                      // warp-uniform
-            // decode the segment's unit k (the CTA's kk-th) from `wds` into A
-            // stage kk & 1, then lane 0 issues its MMA into this warp's accumulator
+            uint32_t wa[QW], wb[QW];
+            // RPW = 1: decode the segment's unit k (the CTA's kk-th) from `wds`
+            // into A stage kk & 1, then one elected lane issues its MMA into
+            // this warp's accumulator
             auto unit = [&](const uint32_t (&wds)[QW], int k, int kq) {
-                const int s = kq & (kAStages - 1), bs = kq & (kBStages - 1);
-                const uint32_t ph = (uint32_t)(kq / kAStages) & 1u, bph = (uint32_t)(kq / kBStages) & 1u;
+                const int s = kq & (AST - 1), bs = kq & (BST - 1);
+                const uint32_t ph = (uint32_t)(kq / AST) & 1u, bph = (uint32_t)(kq / BST) & 1u;
                 // every lane sees the MMA that last read this stage complete before
                 // it stores into the stage
-                if (fail0 || !(kq < kAStages || warp_wait(&aempty[warp * kAStages + s], ph ^ 1u, abort_flag, lane)))
+                if (fail0 || !(kq < AST || warp_wait(&aempty[warp * AST + s], ph ^ 1u, abort_flag, lane)))
                     ok = false;
                 if (!ok) return;
                 uint32_t buf[QW + 1];
@@ -378,23 +438,89 @@ __global__ void __launch_bounds__(kTcThreads, kCtasPerSm) gemm_tc_kernel(TcParam
                     tc_fence_after();
                     const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
                     mma_f16_ss_commit2_elect(dcol, s ? adesc1 : adesc0, bdesc, idesc, k > 0 ? 1u : 0u,
-                                             &aempty[warp * kAStages + s], &bempty[bs]);
+                                             &aempty[warp * AST + s], &bempty[bs]);
                 } else {
                     fail0 = true;                        // warp-uniform: ends the warp's units
                 }
             };
-            uint32_t wa[QW], wb[QW];
+            // RPW = 2: unit k's tile row 0 (words in wa) and tile row 1 (words in
+            // wb) into the warp's one A stage, then both MMAs and the commits
+            // under one election.  The first half of tile row 0 is decoded into
+            // registers before the wait for the previous unit's MMAs.
+            auto unit2 = [&](int k, int kq) {
+                const int bs = kq & (BST - 1);
+                const uint32_t ph = (uint32_t)kq & 1u, bph = (uint32_t)(kq / BST) & 1u;
+                if (fail0) ok = false;
+                if (!ok) return;
+                load_lane_words_checked<BITS>(wb, src + (size_t)k * unit_step + rstep, sib.packed, n_words,
+                                              prm.status);
+                uint32_t buf[QW + 1];
+                buf[0] = __shfl_sync(0xffffffffu, wa[QW - 1], src_prev);
+#pragma unroll
+                for (int t = 0; t < QW; ++t) buf[t + 1] = wa[t];
+                uint32_t stg[4][4], stg_off[4];
+                int n = 0;
+                decode_quarter_chunks<BITS, 0, 4>(buf, soff, prm.two16, [&](uint32_t off, uint32_t w0, uint32_t w1,
+                                                                            uint32_t w2, uint32_t w3) {
+                    stg[n][0] = w0;
+                    stg[n][1] = w1;
+                    stg[n][2] = w2;
+                    stg[n][3] = w3;
+                    stg_off[n] = off;
+                    ++n;
+                });
+                // every lane sees the MMAs that last read the stage complete before it stores
+                if (!(kq < 1 || warp_wait(&aempty[warp], ph ^ 1u, abort_flag, lane))) {
+                    ok = false;
+                    return;
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) sts128(ast0 + stg_off[t], stg[t][0], stg[t][1], stg[t][2], stg[t][3]);
+                decode_quarter_chunks<BITS, 4, 8>(buf, soff, prm.two16, [&](uint32_t off, uint32_t w0, uint32_t w1,
+                                                                            uint32_t w2, uint32_t w3) {
+                    sts128(ast0 + off, w0, w1, w2, w3);
+                });
+                if (k + 1 < nseg)
+                    load_lane_words_checked<BITS>(wa, src + (size_t)(k + 1) * unit_step, sib.packed, n_words,
+                                                  prm.status);
+                buf[0] = __shfl_sync(0xffffffffu, wb[QW - 1], src_prev);
+#pragma unroll
+                for (int t = 0; t < QW; ++t) buf[t + 1] = wb[t];
+                decode_quarter_chunks<BITS, 0, 8>(buf, soff, prm.two16, [&](uint32_t off, uint32_t w0, uint32_t w1,
+                                                                            uint32_t w2, uint32_t w3) {
+                    sts128(ast1 + off, w0, w1, w2, w3);
+                });
+                fence_proxy_async_smem();          // generic-proxy stores -> visible to the tensor core
+                __syncwarp();
+                if (warp_wait(&bfull[bs], bph, abort_flag, lane)) {
+                    tc_fence_after();
+                    const uint64_t bdesc = bdesc0 + (uint64_t)((bs * L::BUNIT) >> 4);
+                    mma2_f16_ss_commit2_elect(dcol, adesc0, bdesc, adesc1, bdesc + (uint64_t)((2 * L::CHUNK) >> 4),
+                                              idesc, k > 0 ? 1u : 0u, &aempty[warp], &bempty[bs]);
+                } else {
+                    fail0 = true;                        // warp-uniform: ends the warp's units
+                }
+            };
             load_lane_words_checked<BITS>(wa, src, sib.packed, n_words, prm.status);
             if (seg == 0) grid_dep_wait();     // weights are never written; y and the workspace after this
-            int k = 0;
-            for (; k + 2 <= nseg; k += 2) {
-                load_lane_words_checked<BITS>(wb, src + (size_t)(k + 1) * unit_step, sib.packed, n_words, prm.status);
-                unit(wa, k, kk + k);
-                if (k + 2 < nseg)
-                    load_lane_words_checked<BITS>(wa, src + (size_t)(k + 2) * unit_step, sib.packed, n_words, prm.status);
-                unit(wb, k + 1, kk + k + 1);
+            if constexpr (RPW == 1) {
+                (void)unit2;
+                int k = 0;
+                for (; k + 2 <= nseg; k += 2) {
+                    load_lane_words_checked<BITS>(wb, src + (size_t)(k + 1) * unit_step, sib.packed, n_words,
+                                                  prm.status);
+                    unit(wa, k, kk + k);
+                    if (k + 2 < nseg)
+                        load_lane_words_checked<BITS>(wa, src + (size_t)(k + 2) * unit_step, sib.packed, n_words,
+                                                      prm.status);
+                    unit(wb, k + 1, kk + k + 1);
+                }
+                if (k < nseg) unit(wa, k, kk + k);
+            } else {
+                static_assert(RPW == 2, "one or two tile rows per warp");
+                (void)unit;
+                for (int k = 0; k < nseg; ++k) unit2(k, kk + k);
             }
-            if (k < nseg) unit(wa, k, kk + k);
             kk += nseg;
             // arrives once every MMA this warp issued has completed -- also after a
             // wait gave up part-way (then it covers the MMAs already in flight)
@@ -573,11 +699,20 @@ int nt_for(int m) { return m <= 16 ? 16 : 32; }
 size_t xt_offset(int G) { (void)G; return align_up(ws_data_off(), 1024); }
 
 // Units of the group (sum over members of blocks x 128-row input blocks).
-long long group_units(const GemmArgs& a)
+// Units of the group at RPW tile rows per warp (128 RPW input rows each).
+long long group_units(const GemmArgs& a, int rpw = 1)
 {
     long long U = 0;
-    for (int i = 0; i < a.nmem; ++i) U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / 128);
+    for (int i = 0; i < a.nmem; ++i) U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / (128 * rpw));
     return U;
+}
+
+// Two tile rows per warp when every member's K_in allows 256-row units.
+int rpw_for(const GemmArgs& a)
+{
+    for (int i = 0; i < a.nmem; ++i)
+        if (a.mem[i].k_in % 256 != 0) return 1;
+    return 2;
 }
 
 // Bytes of rotated input: one k_in x NT fp16 operand per distinct input.
@@ -605,7 +740,8 @@ size_t part_offset(const GemmArgs& a, int NT) { return align_up(xt_offset(a.n_ou
 
 size_t group_ws_bytes(const GemmArgs& a, int NT)
 {
-    // the stream-K partial slots are always reserved (either cut may be chosen)
+    // the stream-K partial slots are always reserved (either cut may be chosen;
+    // counted on 128-row units, the most CTAs any unit size gives)
     const int G = a.n_out / 128;
     return part_offset(a, NT) + (size_t)(sk_ctas(G, group_units(a)) + G) * NT * 128 * sizeof(float);
 }
@@ -643,15 +779,16 @@ struct TcPlan {
 // A cluster size is used only if all G clusters fit at once.
 constexpr double kSegCost = 3.0;
 constexpr double kGlobalRed = 1.2;
-TcPlan choose_plan(int k_in, int n_out, size_t smem)
+TcPlan choose_plan(int k_in, int n_out, size_t smem, int rpw)
 {
     auto kern = cluster_fit_probe_kernel;
-    const int G = n_out / 128, C = k_in / 128;
+    const int G = n_out / 128, C = k_in / (128 * rpw);
     const long long U = (long long)G * C;
+    // costs in 128-row unit decode times
     auto cost_sk = [&](long long P) {
         const long long per = (U + P - 1) / P;
         const double segs = (P % G == 0) ? 1.0 : (double)((per - 1) / C + 2);
-        return (double)per + 0.3 * (double)P / G + kSegCost * segs + kGlobalRed;
+        return (double)(per * rpw) + 0.3 * (double)P / G + kSegCost * segs + kGlobalRed;
     };
     TcPlan best{0, sk_ctas(G, U)};
     double best_cost = cost_sk(best.P);
@@ -684,7 +821,7 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
             continue;
         }
         if (nclusters >= G) {
-            const double cost_cl = (double)((C + S - 1) / S) + 0.2 + 0.05 * S + kSegCost;
+            const double cost_cl = (double)((C + S - 1) / S * rpw) + 0.2 + 0.05 * S + kSegCost;
             if (cost_cl < best_cost) best = TcPlan{S, G * S};
             break;
         }
@@ -692,16 +829,16 @@ TcPlan choose_plan(int k_in, int n_out, size_t smem)
     return best;
 }
 
-template <int BITS, int NT>
-cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
+template <int BITS, int NT, int RPW>
+cudaError_t launch_tc_r(GemmArgs a, cudaStream_t stream)
 {
-    using L = TcLayout<NT>;
+    using L = TcLayout<NT, RPW>;
     // member units and rotated-input offsets of the group
     {
         long long U = 0, xo = 0;
         for (int i = 0; i < a.nmem; ++i) {
             a.mem[i].u0 = U;
-            U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / 128);
+            U += (long long)(a.mem[i].n_out / 128) * (a.mem[i].k_in / (128 * RPW));
             a.mem[i].xt0 = a.shared_x ? 0 : xo;
             xo += (long long)a.mem[i].k_in * NT * 2;
         }
@@ -709,7 +846,7 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
     TcParams prm;
     prm.a = a;
     const int G = a.n_out / 128;
-    prm.U = group_units(a);
+    prm.U = group_units(a, RPW);
     prm.two16 = 0x10000u;
     uint8_t* ws = a.ws;
     prm.status = reinterpret_cast<uint32_t*>(ws);
@@ -739,14 +876,14 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    auto kern = gemm_tc_kernel<BITS, NT>;
+    auto kern = gemm_tc_kernel<BITS, NT, RPW>;
     static std::atomic<int> configured[kMaxDevices];
     e = once_per_device(configured, [&] {
         cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::total);
         if (r == cudaSuccess) r = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         if (r == cudaSuccess)
             r = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     TcLayout<32>::total);
+                                     TcLayout<32, 1>::total);
         if (r == cudaSuccess)
             r = cudaFuncSetAttribute(cluster_fit_probe_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
         return r;
@@ -773,7 +910,7 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
                 }
         }
         if (!hit) {
-            pl = choose_plan(k_in, a.n_out, L::total);
+            pl = choose_plan(k_in, a.n_out, L::total, RPW);
             std::lock_guard<std::mutex> lock(mu);
             cache_key[cache_next] = key;
             cache_val[cache_next] = pl;
@@ -799,6 +936,12 @@ cudaError_t launch_tc_t(GemmArgs a, cudaStream_t stream)
     e = cudaLaunchKernelEx(&cfg, kern, prm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
+}
+
+template <int BITS, int NT>
+cudaError_t launch_tc_t(const GemmArgs& a, cudaStream_t stream)
+{
+    return rpw_for(a) == 2 ? launch_tc_r<BITS, NT, 2>(a, stream) : launch_tc_r<BITS, NT, 1>(a, stream);
 }
 
 }  // namespace

@@ -14,13 +14,16 @@ from gpu_helpers import check_close, to_dev
 pytestmark = pytest.mark.gpu
 
 
-# (k, n, v): v = 1 withholds every rotated-input copy; v = 3 lets each CTA's
-# first two through, so the CTAs with more units have MMAs issued (possibly
-# still in flight) when their wait for the third runs out
-@pytest.mark.parametrize("k,n,v", [(640, 256, 1),        # cluster cut, nothing issued
-                                   (256, 65536, 1),      # stream-K cut, nothing issued
-                                   (5120, 256, 3),       # cluster cut, 4 units per CTA
-                                   (256, 65536, 3)])     # stream-K cut, 3-4 units per CTA
+# (k, n, v): v = 1 withholds every rotated-input copy; v > 1 lets each CTA's
+# first v - 1 through, so the CTAs with more units have MMAs issued (possibly
+# still in flight) when their wait for the next runs out.  K_in a multiple of
+# 256 takes 256-row units (two tile rows per warp), other K_in 128-row units.
+@pytest.mark.parametrize("k,n,v", [(640, 256, 1),        # 128-row units, cluster cut, nothing issued
+                                   (256, 65536, 1),      # 256-row units, stream-K cut, nothing issued
+                                   (5120, 256, 2),       # 256-row units, cluster cut, 2 units per CTA
+                                   (5248, 256, 3),       # 128-row units, 4-5 units per CTA
+                                   (512, 65536, 3),      # 256-row units, stream-K cut, 3-4 units per CTA
+                                   (384, 65536, 3)])     # 128-row units, stream-K cut, 5-6 units per CTA
 def test_withheld_input_times_out_and_reports(oracle_mod, k, n, v):
     import torch
     from gemm_exl3_gemv_b200 import exl3 as ex
