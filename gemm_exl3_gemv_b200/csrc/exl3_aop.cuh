@@ -40,9 +40,12 @@ __device__ __forceinline__ int chan_of_row(int v)
 // row, four 32-bit words), two 16-byte chunks per row.  soff[rb][e]: per-lane
 // byte offset of the chunk holding channels 8e..8e+7 of a row with
 // (row & 1) == rb; row >> 1 selects the 8-row K group (+2048 bytes).
-template <int BITS, int NW, typename Put>
-__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], const uint32_t (&soff)[2][2],
-                                                    uint32_t two16, Put&& put)
+// decode_quarter_chunks does chunks RE0 .. RE1 - 1 only (chunk RE = 2 r + e:
+// row r of the quarter, channels 8e .. 8e + 7), with the same arithmetic and
+// window forms per weight; decode_quarter_to_a does all eight.
+template <int BITS, int RE0, int RE1, int NW, typename Put>
+__device__ __forceinline__ void decode_quarter_chunks(const uint32_t (&buf)[NW], const uint32_t (&soff)[2][2],
+                                                      uint32_t two16, Put&& put)
 {
     auto body = [&](auto R, auto E) {
         constexpr int r = decltype(R)::value, e = decltype(E)::value;
@@ -59,8 +62,15 @@ __device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], c
             pair(std::integral_constant<int, 3>{}));
     };
     [&]<int... RE>(std::integer_sequence<int, RE...>) {
-        (body(std::integral_constant<int, RE / 2>{}, std::integral_constant<int, RE % 2>{}), ...);
-    }(std::make_integer_sequence<int, 8>{});
+        (body(std::integral_constant<int, (RE0 + RE) / 2>{}, std::integral_constant<int, (RE0 + RE) % 2>{}), ...);
+    }(std::make_integer_sequence<int, RE1 - RE0>{});
+}
+
+template <int BITS, int NW, typename Put>
+__device__ __forceinline__ void decode_quarter_to_a(const uint32_t (&buf)[NW], const uint32_t (&soff)[2][2],
+                                                    uint32_t two16, Put&& put)
+{
+    decode_quarter_chunks<BITS, 0, 8>(buf, soff, two16, static_cast<Put&&>(put));
 }
 
 // Per-lane chunk offsets of the layout above for lane (tile j = lane/4,

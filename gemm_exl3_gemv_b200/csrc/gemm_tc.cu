@@ -242,31 +242,6 @@ __device__ __forceinline__ void finish_row(const GemmArgs& a, int g, int mm, con
     finish_row_regs(a, g, mm, z, lane);
 }
 
-// decode_quarter_to_a restricted to its 16-byte chunks RE0 .. RE1 - 1 (chunk
-// RE = 2 r + e: row r of the quarter, channels 8e .. 8e + 7); the same
-// arithmetic and window forms per weight.
-template <int BITS, int RE0, int RE1, int NW, typename Put>
-__device__ __forceinline__ void decode_quarter_chunks(const uint32_t (&buf)[NW], const uint32_t (&soff)[2][2],
-                                                      uint32_t two16, Put&& put)
-{
-    auto body = [&](auto R, auto E) {
-        constexpr int r = decltype(R)::value, e = decltype(E)::value;
-        auto pair = [&](auto Cc) -> uint32_t {
-            constexpr int c = decltype(Cc)::value;
-            constexpr int ia = 16 * r + 8 * e + 2 * c, ib = ia + 1;
-            const uint32_t ma = inst3(window_auto<BITS, ia, (ia + 1) * BITS + 16>(buf, two16));
-            const uint32_t mb = inst3(window_auto<BITS, ib, (ib + 1) * BITS + 16>(buf, two16));
-            return weight_pair_h(ma, mb);
-        };
-        put(soff[r & 1][e] + (r >> 1) * 2048, pair(std::integral_constant<int, 0>{}),
-            pair(std::integral_constant<int, 1>{}), pair(std::integral_constant<int, 2>{}),
-            pair(std::integral_constant<int, 3>{}));
-    };
-    [&]<int... RE>(std::integer_sequence<int, RE...>) {
-        (body(std::integral_constant<int, (RE0 + RE) / 2>{}, std::integral_constant<int, (RE0 + RE) % 2>{}), ...);
-    }(std::make_integer_sequence<int, RE1 - RE0>{});
-}
-
 // Two MMAs into one accumulator (the second always accumulating) and two
 // commits, issued by one elected lane under a single election.
 __device__ __forceinline__ void mma2_f16_ss_commit2_elect(uint32_t d_tmem, uint64_t adesc0, uint64_t bdesc0,
