@@ -232,6 +232,13 @@ class Stack:
             b.append(min(n, int(b[-1] * growth) + 1))
         return list(zip(b[:-1], b[1:]))
 
+    def _out_chunks(self):
+        """{last layer of a chunk: its layer range [a, b)} for the output
+        copies: the input chunks mirrored, so they shrink towards the last
+        layer, whose output goes down alone."""
+        n = len(self.layers)
+        return {n - 1 - a: (n - b, n - a) for a, b in self._copy_chunks()}
+
     def run_e2e(self):
         """One end-to-end step from pinned host buffers: the inputs go up on one
         stream in growing chunks of layers (``_copy_chunks``), the products run
@@ -260,7 +267,7 @@ class Stack:
                 ev = torch.cuda.Event()
                 ev.record(self.s_in)
                 landed[a] = ev
-        out_chunks = {n - 1 - a: (n - b, n - a) for a, b in self._copy_chunks()}   # mirrored
+        out_chunks = self._out_chunks()
         for li in range(n):
             if li in landed:
                 cs.wait_event(landed[li])
